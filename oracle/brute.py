@@ -1,0 +1,58 @@
+"""Second, independent oracle: brute-force dense attention with an explicit 2-D mask.
+
+TEST INFRASTRUCTURE ONLY (tiny shapes). It shares nothing with skiparse_oracle.c: it
+never forms subsequences. Instead it runs ONE dense fp64 attention over the whole
+padded token grid and removes pairs with a 2-D mask
+    M[x, y] = [class(x) == class(y)] and [y is a real token],
+which is what the OSP-Next summary page's 前置知识 (prerequisites) section contrasts
+with Skiparse (a dynamic 2-D mask, which Skiparse's fixed rearrangement avoids). Its
+class rule is written here separately from the C oracle's, from the 核心方法 (core
+method) section: token-wise (h mod P, w mod P), group-wise ((h div P) mod P,
+(w div P) mod P).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def class_grid(Hp: int, Wp: int, P: int, mode: int) -> np.ndarray:
+    h = np.arange(Hp)[:, None]
+    w = np.arange(Wp)[None, :]
+    if mode == 0:
+        ci, cj = h % P, w % P
+    else:
+        ci, cj = (h // P) % P, (w // P) % P
+    return (ci * P + cj).astype(np.int64)
+
+
+def attention(q, k, v, P: int, mode: int) -> np.ndarray:
+    """q, k, v: float64 (B,T,H,W,heads,d). Returns float64 (B,T,H,W,heads,d)."""
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, T, H, W, heads, d = q.shape
+    step = P * P
+    Hp = -(-H // step) * step
+    Wp = -(-W // step) * step
+    pad = ((0, 0), (0, 0), (0, Hp - H), (0, Wp - W), (0, 0), (0, 0))
+    qp, kp, vp = (np.pad(a, pad) for a in (q, k, v))
+    cls = np.broadcast_to(class_grid(Hp, Wp, P, mode), (T, Hp, Wp)).reshape(-1)
+    real = np.zeros((T, Hp, Wp), dtype=bool)
+    real[:, :H, :W] = True
+    real = real.reshape(-1)
+    mask = (cls[:, None] == cls[None, :]) & real[None, :]
+    N = T * Hp * Wp
+    out = np.zeros_like(qp)
+    for b in range(B):
+        for hd in range(heads):
+            Q = qp[b, ..., hd, :].reshape(N, d)
+            K = kp[b, ..., hd, :].reshape(N, d)
+            V = vp[b, ..., hd, :].reshape(N, d)
+            S = (Q[real] @ K.T) / np.sqrt(d)  # real queries only: pads give no output
+            S = np.where(mask[real], S, -np.inf)
+            S = S - S.max(axis=1, keepdims=True)
+            E = np.exp(S)
+            A = E / E.sum(axis=1, keepdims=True)
+            O = np.zeros((N, d))
+            O[real] = A @ V
+            out[b, ..., hd, :] = O.reshape(T, Hp, Wp, d)
+    return out[:, :, :H, :W]

@@ -1,0 +1,34 @@
+"""Compile the CPU oracle (plain C, gcc) into oracle/liboracle.so.
+
+Test infrastructure: building the checker is not using it. Run as
+``python oracle/build.py`` or through ``__graft_entry__.build()``.
+"""
+
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "skiparse_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    deps = [SRC, os.path.join(HERE, "skiparse_oracle.h")]
+    if not force and os.path.exists(LIB):
+        if os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in deps):
+            return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-Wall", "-Wextra",
+           "-fno-fast-math", "-ffp-contract=off", SRC, "-o", tmp, "-lm", "-lpthread"]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose=True))

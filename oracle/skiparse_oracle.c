@@ -1,0 +1,343 @@
+/*
+ * skiparse_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow and deliberately obvious fp64 CPU restatement of Skiparse-2D sparse
+ * attention. Only tests/, the smoke check and the benchmark's CPU-baseline leg use it;
+ * it shares nothing with the CUDA library.
+ *
+ * Method source (cited per function below): the paper.rainbus.top summary of
+ * "OSP-Next: Efficient High-Quality Video Generation with Sparse Sequence Parallelism,
+ * HiF8 Quantization, and Reinforcement Learning", sections 核心方法 (core method) and
+ * 方法步骤详情 (method step details), and the English abstract on the chatpaper.ai page.
+ *
+ * The pages' steps, in their order:
+ *   1. rearrange the (B,T,H,W,C) tokens into P^2 subsequences of length N/P^2
+ *      (token-wise: pixel-unshuffle-like; group-wise: patch-unshuffle-like),
+ *      padding H and W up to the next multiple of P^2 and building an attention mask;
+ *   2. run dense softmax attention inside each subsequence;
+ *   3. rearrange the result back to the original layout.
+ * Readings taken where the pages are silent (each is listed with its reason in the
+ * design notes): group-wise class = ((h div P) mod P, (w div P) mod P); padding goes at
+ * the bottom/right; rearranged layout (B*P^2, n, heads, d) with subsequence index
+ * b*P^2 + ci*P + cj and tokens in (t, r, s) raster order; pad slots hold 0;
+ * softmax scale 1/sqrt(d); no causal mask.
+ */
+#include "skiparse_oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int check_shape(int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || P < 1) return -1;
+    if (mode != ORACLE_TOKEN_WISE && mode != ORACLE_GROUP_WISE) return -1;
+    return 0;
+}
+
+/* Any-resolution rule (方法步骤详情): when H or W is not a multiple of P^2, pad it to
+ * the nearest larger multiple. */
+int oracle_padded_extent(int X, int P) {
+    if (X < 1 || P < 1) return -1;
+    int q = P * P;
+    return ((X + q - 1) / q) * q;
+}
+
+/* Class of one spatial coordinate and its position inside its class's sub-grid.
+ * Token-wise (核心方法: like pixel unshuffle, the H x W map is cut into k x k sub-images,
+ * each sub-image being one sequence): class = x mod P, sub-grid position = x div P.
+ * Group-wise (核心方法: like patch unshuffle, tokens grouped by k x k blocks): the
+ * block index x div P is distributed the token-wise way, so class = (x div P) mod P,
+ * and each block keeps its P tokens together: sub-grid position = (x div P^2)*P + x mod P. */
+int oracle_axis_map(int x, int P, int mode, int* cls, int* sub) {
+    if (x < 0 || P < 1) return -1;
+    if (mode == ORACLE_TOKEN_WISE) {
+        *cls = x % P;
+        *sub = x / P;
+    } else if (mode == ORACLE_GROUP_WISE) {
+        *cls = (x / P) % P;
+        *sub = (x / (P * P)) * P + (x % P);
+    } else {
+        return -1;
+    }
+    return 0;
+}
+
+/* 方法步骤详情: each subsequence is 1/P^2 of the (padded) sequence. */
+long long oracle_subseq_len(int T, int H, int W, int P) {
+    int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    if (T < 1 || Hp < 0 || Wp < 0) return -1;
+    return (long long)T * (Hp / P) * (Wp / P);
+}
+
+/* Step 1 (方法步骤详情): rearrange into P^2 subsequences, pad, and record the mask. */
+int oracle_rearrange(const uint16_t* x, uint16_t* y, uint8_t* valid,
+                     int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    const long long n = (long long)T * R * S;
+    const long long row = (long long)heads * d;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hp; ++h)
+                for (int w = 0; w < Wp; ++w) {
+                    int ci, r, cj, s;
+                    oracle_axis_map(h, P, mode, &ci, &r);
+                    oracle_axis_map(w, P, mode, &cj, &s);
+                    const long long seq = (long long)b * P * P + ci * P + cj;
+                    const long long pos = ((long long)t * R + r) * S + s;
+                    const int real = (h < H) && (w < W);
+                    uint16_t* dst = y + (seq * n + pos) * row;
+                    if (real) {
+                        const long long tok = (((long long)b * T + t) * H + h) * W + w;
+                        for (long long e = 0; e < row; ++e) dst[e] = x[tok * row + e];
+                    } else {
+                        for (long long e = 0; e < row; ++e) dst[e] = 0;
+                    }
+                    if (valid) valid[seq * n + pos] = (uint8_t)real;
+                }
+    return 0;
+}
+
+/* Step 3 (方法步骤详情: rearrange back to the original layout), real tokens only. */
+int oracle_unrearrange(const uint16_t* y, uint16_t* x,
+                       int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    const long long n = (long long)T * R * S;
+    const long long row = (long long)heads * d;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h)
+                for (int w = 0; w < W; ++w) {
+                    int ci, r, cj, s;
+                    oracle_axis_map(h, P, mode, &ci, &r);
+                    oracle_axis_map(w, P, mode, &cj, &s);
+                    const long long seq = (long long)b * P * P + ci * P + cj;
+                    const long long pos = ((long long)t * R + r) * S + s;
+                    const long long tok = (((long long)b * T + t) * H + h) * W + w;
+                    for (long long e = 0; e < row; ++e) x[tok * row + e] = y[(seq * n + pos) * row + e];
+                }
+    return 0;
+}
+
+int oracle_unrearrange_f64(const double* y, double* x,
+                           int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    const long long n = (long long)T * R * S;
+    const long long row = (long long)heads * d;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h)
+                for (int w = 0; w < W; ++w) {
+                    int ci, r, cj, s;
+                    oracle_axis_map(h, P, mode, &ci, &r);
+                    oracle_axis_map(w, P, mode, &cj, &s);
+                    const long long seq = (long long)b * P * P + ci * P + cj;
+                    const long long pos = ((long long)t * R + r) * S + s;
+                    const long long tok = (((long long)b * T + t) * H + h) * W + w;
+                    for (long long e = 0; e < row; ++e) x[tok * row + e] = y[(seq * n + pos) * row + e];
+                }
+    return 0;
+}
+
+/* Step 2: dense softmax attention of one query row over the real keys of its own
+ * subsequence (核心方法: each subsequence attends densely, which is why FlashAttention
+ * runs natively; 方法步骤详情: padded keys are removed by the attention mask).
+ * o = sum_j exp(s_j - m) v_j / sum_j exp(s_j - m), s_j = q.k_j / sqrt(d), m = max_j s_j. */
+static void attend_one(const uint16_t* yq, const uint16_t* yk, const uint16_t* yv,
+                       const uint8_t* valid, long long n, int heads, int d,
+                       long long seq, long long i, int head, double* o, double* score) {
+    const long long row = (long long)heads * d;
+    const uint16_t* q = yq + ((seq * n + i) * heads + head) * d;
+    const double scale = 1.0 / sqrt((double)d);
+    double m = -INFINITY;
+    for (long long j = 0; j < n; ++j) {
+        if (!valid[seq * n + j]) continue;
+        const uint16_t* kj = yk + (seq * n + j) * row + (long long)head * d;
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += bf16_bits_to_double(q[e]) * bf16_bits_to_double(kj[e]);
+        score[j] = acc * scale;
+        if (score[j] > m) m = score[j];
+    }
+    double denom = 0.0;
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    for (long long j = 0; j < n; ++j) {
+        if (!valid[seq * n + j]) continue;
+        const double p = exp(score[j] - m);
+        denom += p;
+        const uint16_t* vj = yv + (seq * n + j) * row + (long long)head * d;
+        for (int e = 0; e < d; ++e) o[e] += p * bf16_bits_to_double(vj[e]);
+    }
+    for (int e = 0; e < d; ++e) o[e] /= denom;
+}
+
+/* ---- thread fan-out over independent query rows ------------------------------- */
+
+typedef struct {
+    const uint16_t *yq, *yk, *yv;
+    const uint8_t* valid;
+    long long n;
+    int heads, d;
+    /* work list: either all (seq, i, head) units, or an explicit unit list */
+    long long nunits;
+    const long long* units;  /* (seq*n + i)*heads + head, or NULL for "unit = index" */
+    double* out;             /* indexed by unit (units == NULL) or by list position */
+    int tid, nthreads;
+} attn_job;
+
+static void* attn_worker(void* arg) {
+    attn_job* jb = (attn_job*)arg;
+    double* score = (double*)malloc(sizeof(double) * (size_t)(jb->n > 0 ? jb->n : 1));
+    if (!score) return (void*)1;
+    for (long long u = jb->tid; u < jb->nunits; u += jb->nthreads) {
+        const long long unit = jb->units ? jb->units[u] : u;
+        const int head = (int)(unit % jb->heads);
+        const long long tokslot = unit / jb->heads;
+        const long long seq = tokslot / jb->n, i = tokslot % jb->n;
+        if (!jb->valid[seq * jb->n + i]) continue;  /* pad queries produce no output */
+        double* o = jb->out + (jb->units ? u : unit) * (long long)jb->d;
+        attend_one(jb->yq, jb->yk, jb->yv, jb->valid, jb->n, jb->heads, jb->d, seq, i, head,
+                   o, score);
+    }
+    free(score);
+    return NULL;
+}
+
+static int run_attention(attn_job proto, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    attn_job* jobs = (attn_job*)malloc(sizeof(attn_job) * (size_t)nthreads);
+    if (!th || !jobs) { free(th); free(jobs); return -2; }
+    int rc = 0, started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = proto;
+        jobs[t].tid = t;
+        jobs[t].nthreads = nthreads;
+        if (pthread_create(&th[t], NULL, attn_worker, &jobs[t]) != 0) { rc = -3; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) {
+        void* ret = NULL;
+        pthread_join(th[t], &ret);
+        if (ret) rc = -2;
+    }
+    free(th);
+    free(jobs);
+    return rc;
+}
+
+int oracle_masked_attention(const uint16_t* yq, const uint16_t* yk, const uint16_t* yv,
+                            const uint8_t* valid, double* yo, long long nseq, long long n,
+                            int heads, int d, int nthreads) {
+    if (nseq < 1 || n < 1 || heads < 1 || d < 1) return -1;
+    attn_job jb;
+    memset(&jb, 0, sizeof jb);
+    jb.yq = yq; jb.yk = yk; jb.yv = yv; jb.valid = valid;
+    jb.n = n; jb.heads = heads; jb.d = d;
+    jb.nunits = nseq * n * heads;
+    jb.units = NULL;
+    jb.out = yo;
+    return run_attention(jb, nthreads);
+}
+
+typedef struct {
+    uint16_t *yq, *yk, *yv;
+    uint8_t* valid;
+} rearranged;
+
+static void free_rearranged(rearranged* r) {
+    free(r->yq); free(r->yk); free(r->yv); free(r->valid);
+}
+
+static int rearrange_all(const uint16_t* q, const uint16_t* k, const uint16_t* v, rearranged* r,
+                         int B, int T, int H, int W, int heads, int d, int P, int mode,
+                         long long* n_out) {
+    const long long n = oracle_subseq_len(T, H, W, P);
+    const long long nseq = (long long)B * P * P;
+    const size_t elems = (size_t)(nseq * n * heads * d);
+    memset(r, 0, sizeof *r);
+    r->yq = (uint16_t*)malloc(elems * 2);
+    r->yk = (uint16_t*)malloc(elems * 2);
+    r->yv = (uint16_t*)malloc(elems * 2);
+    r->valid = (uint8_t*)malloc((size_t)(nseq * n));
+    if (!r->yq || !r->yk || !r->yv || !r->valid) { free_rearranged(r); return -2; }
+    oracle_rearrange(q, r->yq, r->valid, B, T, H, W, heads, d, P, mode);
+    oracle_rearrange(k, r->yk, NULL, B, T, H, W, heads, d, P, mode);
+    oracle_rearrange(v, r->yv, NULL, B, T, H, W, heads, d, P, mode);
+    *n_out = n;
+    return 0;
+}
+
+int oracle_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, double* out,
+                    int B, int T, int H, int W, int heads, int d, int P, int mode,
+                    int nthreads) {
+    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+    rearranged r;
+    long long n = 0;
+    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
+    if (rc) return rc;
+    const long long nseq = (long long)B * P * P;
+    double* yo = (double*)calloc((size_t)(nseq * n * heads * d), sizeof(double));
+    if (!yo) { free_rearranged(&r); return -2; }
+    rc = oracle_masked_attention(r.yq, r.yk, r.yv, r.valid, yo, nseq, n, heads, d, nthreads);
+    if (!rc) rc = oracle_unrearrange_f64(yo, out, B, T, H, W, heads, d, P, mode);
+    free(yo);
+    free_rearranged(&r);
+    return rc;
+}
+
+int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const long long* rows, long long nrows, double* out_rows,
+                         int B, int T, int H, int W, int heads, int d, int P, int mode,
+                         int nthreads) {
+    if (check_shape(B, T, H, W, heads, d, P, mode) || nrows < 0) return -1;
+    const long long ntok = (long long)B * T * H * W;
+    for (long long i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= ntok * heads) return -1;
+    rearranged r;
+    long long n = 0;
+    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
+    if (rc) return rc;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    long long* units = (long long*)malloc(sizeof(long long) * (size_t)(nrows > 0 ? nrows : 1));
+    if (!units) { free_rearranged(&r); return -2; }
+    /* map each requested original (token, head) to its subsequence slot */
+    for (long long i = 0; i < nrows; ++i) {
+        const int head = (int)(rows[i] % heads);
+        long long tok = rows[i] / heads;
+        const int w = (int)(tok % W); tok /= W;
+        const int h = (int)(tok % H); tok /= H;
+        const int t = (int)(tok % T);
+        const int b = (int)(tok / T);
+        int ci, rr, cj, ss;
+        oracle_axis_map(h, P, mode, &ci, &rr);
+        oracle_axis_map(w, P, mode, &cj, &ss);
+        const long long seq = (long long)b * P * P + ci * P + cj;
+        const long long pos = ((long long)t * R + rr) * S + ss;
+        units[i] = (seq * n + pos) * heads + head;
+    }
+    attn_job jb;
+    memset(&jb, 0, sizeof jb);
+    jb.yq = r.yq; jb.yk = r.yk; jb.yv = r.yv; jb.valid = r.valid;
+    jb.n = n; jb.heads = heads; jb.d = d;
+    jb.nunits = nrows;
+    jb.units = units;
+    jb.out = out_rows;
+    rc = nrows > 0 ? run_attention(jb, nthreads) : 0;
+    free(units);
+    free_rearranged(&r);
+    return rc;
+}
