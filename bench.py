@@ -1,0 +1,441 @@
+#!/usr/bin/env python3
+"""Benchmark of the Skiparse-2D attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 720p] [--impl ours|reference]
+
+One step = one fused skiparse2d_attn_fwd call (class rearrange + pad mask + per-class dense
+attention + inverse rearrange, one kernel launch) over the whole synthetic workload; the
+step alternates token-wise and group-wise mode, as the layers of the model do. Inputs are
+seeded N(0,1) bf16 tensors larger than L2, resident in HBM when timing starts. `value` is
+TFLOP/s by the padded formula 4*N*(N/P^2)*d*heads*B, N = T*Hp*Wp, summed over ranks.
+
+Under torchrun (N > 1) every rank runs its own independent copy of the workload (the path
+has no exchange step: (b, class, head) units are independent), timing is the max over
+ranks, and `scaling` is "weak".
+
+--impl reference times the CPU oracle (the only reference this method has: no reference
+implementation is shipped) on a bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import skiparse_synth as synth  # noqa: E402
+
+METRIC = "Skiparse-2D attn fwd TFLOP/s and % BF16 peak at 720p P=2; ms/layer vs P=1 dense"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the attention kernel, from an ncu capture, keyed by the hash of
+# the kernel sources it was captured on (a changed kernel reports null until re-captured).
+KNOWN_TRAFFIC = {}
+
+ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
+                "fixed_pattern_sparse_b200/csrc/ptx_sm100.cuh",
+                "fixed_pattern_sparse_b200/csrc/skiparse_internal.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def padded(X, P):
+    return -(-X // (P * P)) * (P * P)
+
+
+def flops_padded(w) -> float:
+    N = w.T * padded(w.H, w.P) * padded(w.W, w.P)
+    return 4.0 * N * (N / (w.P * w.P)) * w.d * w.heads * w.B
+
+
+def class_lens(w, mode):
+    import fixed_pattern_sparse_b200 as fps
+    return [fps.class_len(w.T, w.H, w.W, w.P, mode, ci, cj) for ci in range(w.P) for cj in range(w.P)]
+
+
+def flops_real(w, mode) -> float:
+    return sum(4.0 * n * n * w.d * w.heads * w.B for n in class_lens(w, mode))
+
+
+def describe(w) -> str:
+    return (f"{w.name} latent B={w.B} T={w.T} H={w.H} W={w.W} heads={w.heads} d={w.d} P={w.P} "
+            f"(padded {padded(w.H, w.P)}x{padded(w.W, w.P)})")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        ident = None
+        try:
+            ident = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        if ident is None:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ident = vis.split(",")[device_index] if vis else str(device_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = []
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[4], parts[6:10]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "samples": len(inside), "power_w_max": max(float(r[3]) for r in inside if r[3].replace('.', '', 1).isdigit())
+                if any(r[3].replace('.', '', 1).isdigit() for r in inside) else None,
+                "reasons": reasons}
+
+
+# ------------------------------------------------------------------------ distributed
+
+def dist_setup(gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != gpus:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    return rank, world, local
+
+
+def init_pg(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.distributed.init_process_group(backend, timeout=_dt.timedelta(seconds=300))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample_rows(w, mode, nrows: int, group: int = 0) -> np.ndarray:
+    """`nrows` query rows (token*heads + head) of one (class, head) group, for timing the
+    oracle: all real tokens of class `group % P^2`, head `group // P^2`."""
+    import oracle
+    q2 = w.P * w.P
+    c, head = group % q2, (group // q2) % w.heads
+    toks = []
+    for t in range(w.T):
+        for h in range(w.H):
+            ci, _ = oracle.axis_map(h, w.P, mode)
+            for x in range(w.W):
+                cj, _ = oracle.axis_map(x, w.P, mode)
+                if ci * w.P + cj == c:
+                    toks.append((t * w.H + h) * w.W + x)
+    toks = np.array(toks, dtype=np.int64)
+    pick = np.linspace(0, len(toks) - 1, num=min(nrows, len(toks))).astype(np.int64)
+    return toks[pick] * w.heads + head
+
+
+def time_oracle(w, q, k, v, mode, target_s: float, nthreads: int):
+    """Times the oracle on a bounded sample sized to about target_s seconds of CPU work.
+    Returns (TFLOP/s, seconds, rows, description)."""
+    import oracle
+    n_c = max(class_lens(w, mode))
+    per_row = 4.0 * n_c * w.d
+    rows = oracle_sample_rows(w, mode, max(nthreads, 8))
+    t = time.perf_counter()
+    oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
+    dt = time.perf_counter() - t
+    nrows = int(min(max(len(rows) * target_s / max(dt, 1e-3), nthreads), 200000))
+    rows = oracle_sample_rows(w, mode, nrows)
+    t = time.perf_counter()
+    oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
+    dt = time.perf_counter() - t
+    flops = per_row * len(rows)
+    desc = (f"{len(rows)} query rows of one (class, head) subsequence of the {w.name} workload "
+            f"({MODE_NAME[mode]}), each attending over its class's ~{n_c} real keys; the oracle's "
+            f"per-subsequence gather included")
+    return flops / dt / 1e12, dt, len(rows), desc
+
+
+MODE_NAME = synth.MODE_NAMES
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_pg(world, "nccl")
+    import fixed_pattern_sparse_b200 as fps
+
+    w = synth.WORKLOADS[args.workload]
+    modes = [0, 1] if args.mode == "both" else [0 if args.mode == "token" else 1]
+    if w.P == 1:
+        modes = [0]
+    q, k, v = synth.qkv(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qd)
+    fl = flops_padded(w)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, modes[i % len(modes)], out=out)
+
+    for i in range(args.warmup):
+        step(i)
+    if fps.get_device_status() != 0:
+        raise SystemExit("device status error during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(world)
+    clk = clocks.stop(t_wall0, t_wall1)
+    if fps.get_device_status() != 0:
+        raise SystemExit("device status error in the timed region")
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = starts[0].elapsed_time(ends[-1])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_step = total_ms / args.steps
+    value = fl * args.steps * world / (total_ms / 1e3) / 1e12
+    by_mode = {MODE_NAME[m]: statistics.mean(per_launch[i] for i in range(args.steps) if i % len(modes) == j)
+               for j, m in enumerate(modes)}
+
+    peaks, peak_src = load_peaks()
+    mean_launch_s = statistics.mean(per_launch) / 1e3
+    achieved = fl / mean_launch_s / 1e12
+    peak = float(peaks["bf16_tflops"])
+    roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": KNOWN_TRAFFIC.get(kernel_hash()),
+            "kernel": "skiparse_attn_fwd_kernel<128>",
+            "peak_source": f"{peak_src} burst cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)",
+            "frac_of_sustained": round(achieved / float(peaks.get("bf16_tflops_sustained", peak)), 4),
+            "flop_per_launch": fl}
+
+    # end to end through the public host API: pinned host in, pinned host out
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+        oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        staging = fps.HostStaging(q.shape, device=dev)
+        for i in range(2):
+            fps.attn_fwd_from_host(qh, kh, vh, w.P, modes[i % len(modes)], oh, staging)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(stream)
+        for i in range(args.e2e_steps):
+            fps.attn_fwd_from_host(qh, kh, vh, w.P, modes[i % len(modes)], oh, staging)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": round(fl * args.e2e_steps * world / (e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2,
+               "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps}
+        del staging, qh, kh, vh, oh
+
+    # P = 1 dense attention at the same shape on the same kernel: ms/layer and sparse speedup
+    dense = None
+    if not args.no_dense and w.P > 1:
+        wd = synth.custom(w.B, w.T, w.H, w.W, w.heads, w.d, 1, name=w.name + "_p1")
+        for _ in range(2):
+            fps.skiparse2d_attn_fwd(qd, kd, vd, 1, 0, out=out)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(args.dense_steps):
+            fps.skiparse2d_attn_fwd(qd, kd, vd, 1, 0, out=out)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        dms = d0.elapsed_time(d1) / args.dense_steps
+        dense = {"ms_per_layer_p1": round(dms, 3), "tflops_p1": round(flops_padded(wd) / (dms / 1e3) / 1e12, 1),
+                 "sparse_speedup": round(dms / statistics.mean(per_launch), 3)}
+        if fps.get_device_status() != 0:
+            raise SystemExit("device status error in the dense comparison")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nth = oracle.default_threads()
+        val, dt, nrows, desc = time_oracle(w, q, k, v, modes[0], args.cpu_seconds, nth)
+        cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": nth, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        real = {MODE_NAME[m]: round(flops_real(w, m) / (by_mode[MODE_NAME[m]] / 1e3) / 1e12, 1) for m in modes}
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16 (no dataset)",
+            "config": {"workload": describe(w),
+                       "modes": "alternating " + " / ".join(MODE_NAME[m] for m in modes) + " per step",
+                       "flop_formula": "4*N*(N/P^2)*d*heads*B with N = T*Hp*Wp (padded)",
+                       "l2": f"inputs larger than L2 ({3 * q.numel() * 2 / 1e9:.2f} GB of q/k/v per step), no flush",
+                       "parallelism": f"{world} independent replica(s), one per GPU, no collective"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "ms_per_layer": {k_: round(v_, 3) for k_, v_ in by_mode.items()},
+            "tflops_real_pairs": real,
+            "dense_p1": dense,
+            "kernel_hash": kernel_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+# --------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    modes = [0, 1] if args.mode == "both" else [0 if args.mode == "token" else 1]
+    if w.P == 1:
+        modes = [0]
+    q, k, v = synth.qkv(w)
+    nth = oracle.default_threads()
+    n_c = {m: max(class_lens(w, m)) for m in modes}
+    # size one step's sample so that all warm-up + timed steps take a few minutes
+    budget_per_step = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = {}
+    for m in modes:
+        probe = oracle_sample_rows(w, m, max(nth, 8))
+        t = time.perf_counter()
+        oracle.attn_fwd_rows(q, k, v, probe, w.P, m, nth)
+        dt = time.perf_counter() - t
+        rows[m] = oracle_sample_rows(w, m, int(max(nth, len(probe) * budget_per_step / max(dt, 1e-3))))
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        m = modes[i % len(modes)]
+        t = time.perf_counter()
+        oracle.attn_fwd_rows(q, k, v, rows[m], w.P, m, nth)
+        dt = time.perf_counter() - t
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(4.0 * n_c[m] * w.d * len(rows[m]))
+    value = sum(flops) / sum(times) / 1e12
+    sample = (f"per step: {len(rows[modes[0]])} query rows of one (class, head) subsequence of the "
+              f"{w.name} workload, each over its class's ~{n_c[modes[0]]} real keys (fp64 oracle)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16 (no dataset)",
+            "config": {"workload": describe(w),
+                       "modes": "alternating " + " / ".join(MODE_NAME[m] for m in modes) + " per step",
+                       "flop_formula": "4 * (real keys of the class) * d per sampled query row"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nth, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="720p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--mode", choices=["both", "token", "group"], default="both")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--dense-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

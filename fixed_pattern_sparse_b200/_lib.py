@@ -1,0 +1,63 @@
+"""ctypes loader for libskiparse.so (the C ABI in include/skiparse.h).
+
+The library is built in-tree by ``python -m fixed_pattern_sparse_b200.build``. There is no
+fallback: if the library is missing or fails to load, importing the binding raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libskiparse.so")
+
+# Every symbol include/skiparse.h declares, with (restype, argtypes).
+_I, _LL, _ULL, _VP, _CP = ctypes.c_int, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_char_p
+SIGNATURES = {
+    "skiparse2d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse_rearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse_unrearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse_rearranged_numel": (_LL, [_I] * 7),
+    "skiparse_padded_extent": (_I, [_I, _I]),
+    "skiparse_subseq_len": (_LL, [_I] * 4),
+    "skiparse_class_len": (_LL, [_I] * 7),
+    "skiparse_get_device_status": (_I, [_VP]),
+    "skiparse_status_string": (_CP, [_I]),
+    "skiparse_version": (_CP, []),
+    "skiparse_set_wait_limit_ns": (_ULL, [_ULL]),
+    "skiparse_debug_inject_fault": (_I, [_I]),
+}
+
+STATUS = {0: "SKIPARSE_OK", 1: "SKIPARSE_ERR_INVALID_ARG", 2: "SKIPARSE_ERR_UNSUPPORTED",
+          3: "SKIPARSE_ERR_MISALIGNED", 4: "SKIPARSE_ERR_CUDA", 5: "SKIPARSE_ERR_TIMEOUT"}
+
+
+class SkiparseError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m fixed_pattern_sparse_b200.build` "
+                "(there is no CPU or library fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def check(code: int, what: str) -> None:
+    if code != 0:
+        raise SkiparseError(code, what)

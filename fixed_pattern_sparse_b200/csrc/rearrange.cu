@@ -1,0 +1,114 @@
+// rearrange.cu -- standalone Skiparse rearrange and inverse rearrange for B200 (sm_100a).
+//
+// Summary page of OSP-Next, 方法步骤详情 (method step details): the (B,T,H,W,C) tokens are
+// rearranged into P^2 subsequences of length N/P^2 (padding H and W up to multiples of P^2),
+// and the attention result is rearranged back to the original layout. Both directions are a
+// permutation of whole token rows of heads*d bf16 values (contiguous in both layouts), so
+// the kernels are pure HBM copies: one warp moves one row with 16-byte loads and stores,
+// several chunks in flight per lane; pad rows of the rearranged tensor are written as zero.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "skiparse_internal.cuh"
+
+namespace skiparse {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4* p, const uint4& v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// forward = true : row is a slot (seq*n + pos) of the rearranged tensor.
+// forward = false: row is a token ((b*T + t)*H + h)*W + w of the original tensor.
+template <bool kForward>
+__global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const RearrangeParams p) {
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = (static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * kThreads) >> 5;
+    const int q2 = p.P * p.P;
+    const uint4* src = static_cast<const uint4*>(p.src);
+    uint4* dst = static_cast<uint4*>(p.dst);
+    for (long long row = warp0; row < p.nrows; row += nwarps) {
+        long long src_row;
+        bool real = true;
+        if (kForward) {
+            const long long seq = row / p.n;
+            const long long pos = row - seq * p.n;
+            const int b = static_cast<int>(seq / q2);
+            const int c = static_cast<int>(seq - static_cast<long long>(b) * q2);
+            const int s = static_cast<int>(pos % p.S);
+            const long long tr = pos / p.S;
+            const int r = static_cast<int>(tr % p.R);
+            const int t = static_cast<int>(tr / p.R);
+            const int h = axis_coord(r, c / p.P, p.P, p.mode);
+            const int w = axis_coord(s, c % p.P, p.P, p.mode);
+            real = h < p.H && w < p.W;
+            src_row = ((static_cast<long long>(b) * p.T + t) * p.H + h) * p.W + w;
+        } else {
+            long long tok = row;
+            const int w = static_cast<int>(tok % p.W);
+            tok /= p.W;
+            const int h = static_cast<int>(tok % p.H);
+            tok /= p.H;
+            const int t = static_cast<int>(tok % p.T);
+            const int b = static_cast<int>(tok / p.T);
+            int ci, r, cj, s;
+            axis_class(h, p.P, p.mode, ci, r);
+            axis_class(w, p.P, p.mode, cj, s);
+            const long long seq = static_cast<long long>(b) * q2 + ci * p.P + cj;
+            src_row = seq * p.n + (static_cast<long long>(t) * p.R + r) * p.S + s;
+        }
+        const uint4* s_row = src + src_row * p.row_chunks;
+        uint4* d_row = dst + row * p.row_chunks;
+        for (int k = lane; k < p.row_chunks; k += 32 * kUnroll) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int idx = k + 32 * u;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (real && idx < p.row_chunks) v[u] = ld_stream(s_row + idx);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int idx = k + 32 * u;
+                if (idx < p.row_chunks) st_stream(d_row + idx, v[u]);
+            }
+        }
+    }
+}
+
+}  // namespace
+
+int launch_rearrange(const RearrangeParams& p, bool forward, void* stream) {
+    if (p.nrows <= 0) return static_cast<int>(cudaSuccess);
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long warps_needed = p.nrows;
+    const long long blocks_needed = (warps_needed * 32 + kThreads - 1) / kThreads;
+    const long long max_blocks = static_cast<long long>(sms) * 8;  // 8 x 256 threads per SM
+    const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (forward)
+        skiparse_rearrange_kernel<true><<<blocks, kThreads, 0, st>>>(p);
+    else
+        skiparse_rearrange_kernel<false><<<blocks, kThreads, 0, st>>>(p);
+    return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace skiparse

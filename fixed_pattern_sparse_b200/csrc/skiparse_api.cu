@@ -1,0 +1,249 @@
+// skiparse_api.cu -- the C ABI of libskiparse.so (declared in include/skiparse.h):
+// argument validation, Skiparse-2D geometry, TMA tensor-map encoding, kernel launch and the
+// per-device status word. Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/skiparse.h"
+#include "skiparse_internal.cuh"
+
+namespace {
+
+using skiparse::Geometry;
+
+__device__ int g_skiparse_status = 0;  // one error word per device
+
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_fault{0};
+
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+int padded(int X, int P) { return ((X + P * P - 1) / (P * P)) * (P * P); }
+
+// Validates the shared shape arguments and fills the geometry. Returns a status code.
+int make_geometry(int B, int T, int H, int W, int heads, int d, int P, int mode, Geometry& g) {
+    if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || P < 1) return SKIPARSE_ERR_INVALID_ARG;
+    if (mode != SKIPARSE_TOKEN_WISE && mode != SKIPARSE_GROUP_WISE) return SKIPARSE_ERR_INVALID_ARG;
+    if (P > skiparse::kMaxP) return SKIPARSE_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64 && d != 128) return SKIPARSE_ERR_UNSUPPORTED;
+    const long long q2 = static_cast<long long>(P) * P;
+    if (H > (1 << 24) || W > (1 << 24)) return SKIPARSE_ERR_UNSUPPORTED;
+    const long long Hp = (H + q2 - 1) / q2 * q2, Wp = (W + q2 - 1) / q2 * q2;
+    const long long rows = static_cast<long long>(B) * T * H * W * heads;       // original rows
+    const long long prow = static_cast<long long>(B) * T * Hp * Wp * heads;     // rearranged rows
+    if (rows >= (1ll << 31) || prow >= (1ll << 31)) return SKIPARSE_ERR_UNSUPPORTED;
+    if (heads > 65535 || B * q2 > 65535) return SKIPARSE_ERR_UNSUPPORTED;
+    g.B = B; g.T = T; g.H = H; g.W = W; g.heads = heads; g.d = d; g.P = P; g.mode = mode;
+    g.Hp = static_cast<int>(Hp);
+    g.Wp = static_cast<int>(Wp);
+    g.R = g.Hp / P;
+    g.S = g.Wp / P;
+    g.n = static_cast<long long>(T) * g.R * g.S;
+    for (int c = 0; c < skiparse::kMaxP; ++c) {
+        g.Rc[c] = 0;
+        g.Sc[c] = 0;
+    }
+    for (int c = 0; c < P; ++c) {
+        for (int r = 0; r < g.R; ++r)
+            if (skiparse::axis_coord(r, c, P, mode) < H) ++g.Rc[c];
+        for (int s = 0; s < g.S; ++s)
+            if (skiparse::axis_coord(s, c, P, mode) < W) ++g.Sc[c];
+    }
+    return SKIPARSE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t abytes, const void* b, size_t bbytes) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bbytes && b0 < a0 + abytes;
+}
+
+int* status_ptr() {
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_skiparse_status) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return p;
+}
+
+// 2-D view (rows = tokens*heads, cols = d) of a (…, heads, d) bf16 tensor, box = one row x
+// (64 or 32) columns, swizzled so the tile lands in the UMMA canonical K-major layout.
+int encode_rows_map(CUtensorMap* map, const void* base, long long rows, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return SKIPARSE_ERR_CUDA;
+    const int box_cols = d >= 64 ? 64 : 32;
+    const CUtensorMapSwizzle sw = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* skiparse_status_string(int status) {
+    switch (status) {
+        case SKIPARSE_OK: return "SKIPARSE_OK";
+        case SKIPARSE_ERR_INVALID_ARG: return "SKIPARSE_ERR_INVALID_ARG";
+        case SKIPARSE_ERR_UNSUPPORTED: return "SKIPARSE_ERR_UNSUPPORTED";
+        case SKIPARSE_ERR_MISALIGNED: return "SKIPARSE_ERR_MISALIGNED";
+        case SKIPARSE_ERR_CUDA: return "SKIPARSE_ERR_CUDA";
+        case SKIPARSE_ERR_TIMEOUT: return "SKIPARSE_ERR_TIMEOUT";
+        default: return "SKIPARSE_ERR_UNKNOWN";
+    }
+}
+
+const char* skiparse_version(void) { return "skiparse-b200 0.1 (sm_100a, tcgen05)"; }
+
+int skiparse_padded_extent(int X, int P) {
+    if (X < 1 || P < 1 || P > skiparse::kMaxP) return -1;
+    return padded(X, P);
+}
+
+long long skiparse_subseq_len(int T, int H, int W, int P) {
+    if (T < 1 || H < 1 || W < 1 || P < 1 || P > skiparse::kMaxP) return -1;
+    return static_cast<long long>(T) * (padded(H, P) / P) * (padded(W, P) / P);
+}
+
+long long skiparse_class_len(int T, int H, int W, int P, int mode, int ci, int cj) {
+    Geometry g;
+    if (make_geometry(1, T, H, W, 1, 32, P, mode, g) != SKIPARSE_OK) return -1;
+    if (ci < 0 || cj < 0 || ci >= P || cj >= P) return -1;
+    return static_cast<long long>(T) * g.Rc[ci] * g.Sc[cj];
+}
+
+long long skiparse_rearranged_numel(int B, int T, int H, int W, int heads, int d, int P) {
+    Geometry g;
+    if (make_geometry(B, T, H, W, heads, d, P, SKIPARSE_TOKEN_WISE, g) != SKIPARSE_OK) return -1;
+    return static_cast<long long>(B) * P * P * g.n * heads * d;
+}
+
+unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns) {
+    return g_wait_limit_ns.exchange(ns == 0 ? kDefaultWaitNs : ns);
+}
+
+int skiparse_debug_inject_fault(int kind) {
+    if (kind != 0 && kind != 1) return SKIPARSE_ERR_INVALID_ARG;
+    g_fault.store(kind);
+    return SKIPARSE_OK;
+}
+
+int skiparse_get_device_status(skiparse_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return SKIPARSE_ERR_CUDA;
+    }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_skiparse_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return SKIPARSE_ERR_CUDA;
+    }
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_skiparse_status, &zero, sizeof(int)) != cudaSuccess) {
+            cudaGetLastError();
+            return SKIPARSE_ERR_CUDA;
+        }
+    }
+    return v;
+}
+
+int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int T,
+                        int H, int W, int heads, int d, int P, int mode, skiparse_stream_t stream) {
+    if (!q || !k || !v || !out) return SKIPARSE_ERR_INVALID_ARG;
+    Geometry g;
+    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    if (st != SKIPARSE_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SKIPARSE_ERR_MISALIGNED;
+    const long long rows = static_cast<long long>(B) * T * H * W * heads;
+    const size_t bytes = static_cast<size_t>(rows) * d * 2;
+    if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
+        return SKIPARSE_ERR_INVALID_ARG;
+    alignas(64) CUtensorMap tq, tk, tv;
+    if (encode_rows_map(&tq, q, rows, d) || encode_rows_map(&tk, k, rows, d) ||
+        encode_rows_map(&tv, v, rows, d))
+        return SKIPARSE_ERR_CUDA;
+    skiparse::AttnParams p{};
+    p.out = static_cast<uint16_t*>(out);
+    p.status = status_ptr();
+    if (!p.status) return SKIPARSE_ERR_CUDA;
+    p.T = T; p.H = H; p.W = W; p.heads = heads; p.P = P; p.mode = mode;
+    for (int c = 0; c < skiparse::kMaxP; ++c) {
+        p.Rc[c] = g.Rc[c];
+        p.Sc[c] = g.Sc[c];
+    }
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.fault = g_fault.exchange(0);
+    const int e = skiparse::launch_attn_fwd(&tq, &tk, &tv, p, g, stream);
+    return e == 0 ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
+}
+
+static int rearrange_common(const void* src, void* dst, int B, int T, int H, int W, int heads,
+                            int d, int P, int mode, skiparse_stream_t stream, bool forward) {
+    if (!src || !dst) return SKIPARSE_ERR_INVALID_ARG;
+    Geometry g;
+    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    if (st != SKIPARSE_OK) return st;
+    if (!aligned16(src) || !aligned16(dst)) return SKIPARSE_ERR_MISALIGNED;
+    const long long row_bytes = static_cast<long long>(heads) * d * 2;
+    const long long ntok = static_cast<long long>(B) * T * H * W;
+    const long long nslot = static_cast<long long>(B) * P * P * g.n;
+    const size_t orig_bytes = static_cast<size_t>(ntok * row_bytes);
+    const size_t rear_bytes = static_cast<size_t>(nslot * row_bytes);
+    if (forward ? overlaps(src, orig_bytes, dst, rear_bytes) : overlaps(src, rear_bytes, dst, orig_bytes))
+        return SKIPARSE_ERR_INVALID_ARG;
+    skiparse::RearrangeParams p{};
+    p.src = src;
+    p.dst = dst;
+    p.B = B; p.T = T; p.H = H; p.W = W; p.P = P; p.mode = mode; p.R = g.R; p.S = g.S;
+    p.n = g.n;
+    p.row_chunks = static_cast<int>(row_bytes / 16);
+    p.nrows = forward ? nslot : ntok;
+    const int e = skiparse::launch_rearrange(p, forward, stream);
+    return e == 0 ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
+}
+
+int skiparse_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d, int P,
+                       int mode, skiparse_stream_t stream) {
+    return rearrange_common(x, y, B, T, H, W, heads, d, P, mode, stream, true);
+}
+
+int skiparse_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
+                         int P, int mode, skiparse_stream_t stream) {
+    return rearrange_common(y, x, B, T, H, W, heads, d, P, mode, stream, false);
+}
+
+}  // extern "C"

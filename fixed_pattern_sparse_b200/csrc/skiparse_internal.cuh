@@ -1,0 +1,77 @@
+// skiparse_internal.cuh -- geometry and launch parameters shared by the C-ABI host code and the
+// sm_100a kernels of libskiparse.so.
+//
+// Geometry of Skiparse-2D (summary page of OSP-Next, sections 核心方法 and 方法步骤详情):
+//   class of a spatial coordinate x along one axis:
+//     token-wise  : x mod P                 (pixel-unshuffle-like)
+//     group-wise  : (x div P) mod P         (patch-unshuffle-like)
+//   position inside the class's sub-grid along that axis:
+//     token-wise  : x div P
+//     group-wise  : (x div P^2)*P + x mod P (each P-wide block stays together)
+//   H and W are padded at the end to the next multiple of P^2 (any-resolution rule).
+// Because the coordinate map is increasing in the sub-grid position, the real (unpadded)
+// tokens of a class occupy a prefix [0, Rc) x [0, Sc) of its sub-grid; the kernels enumerate
+// only those, so the pad-key mask reduces to the ragged tail of the last key tile.
+#pragma once
+
+#include <cstdint>
+
+namespace skiparse {
+
+constexpr int kMaxP = 8;
+
+// Spatial coordinate of sub-grid position `sub` of class `cls` along one axis.
+__host__ __device__ __forceinline__ int axis_coord(int sub, int cls, int P, int mode) {
+    return mode == 0 ? cls + P * sub : (sub / P) * P * P + cls * P + (sub % P);
+}
+
+// Class and sub-grid position of spatial coordinate x along one axis.
+__host__ __device__ __forceinline__ void axis_class(int x, int P, int mode, int& cls, int& sub) {
+    if (mode == 0) {
+        cls = x % P;
+        sub = x / P;
+    } else {
+        cls = (x / P) % P;
+        sub = (x / (P * P)) * P + x % P;
+    }
+}
+
+struct Geometry {
+    int B, T, H, W, heads, d, P, mode;
+    int Hp, Wp;        // padded extents
+    int R, S;          // padded sub-grid extents Hp/P, Wp/P
+    long long n;       // padded subsequence length T*R*S
+    int Rc[kMaxP];     // real sub-grid rows of class row ci
+    int Sc[kMaxP];     // real sub-grid columns of class column cj
+};
+
+// Parameters of the fused attention kernel (plain values only; tensor maps are separate).
+struct AttnParams {
+    uint16_t* out;                 // bf16 bits, (B,T,H,W,heads,d)
+    int* status;                   // device error word
+    int T, H, W, heads, P, mode;
+    int Rc[kMaxP], Sc[kMaxP];
+    float scale_log2;              // log2(e)/sqrt(d)
+    unsigned long long wait_limit_ns;
+    int fault;                     // test hook: 1 = under-deliver the first K tile
+};
+
+struct RearrangeParams {
+    const void* src;
+    void* dst;
+    int B, T, H, W, P, mode, R, S;
+    long long n;          // padded subsequence length
+    int row_chunks;       // 16-byte chunks per token row (heads*d*2/16)
+    long long nrows;      // rows to write: B*P*P*n (rearrange) or B*T*H*W (unrearrange)
+};
+
+// Status codes (mirror include/skiparse.h).
+enum : int { kOk = 0, kErrTimeout = 5 };
+
+// Launchers (defined in the kernel translation units). They return the cudaError_t as int.
+int launch_attn_fwd(const void* tmap_q, const void* tmap_k, const void* tmap_v,
+                    const AttnParams& p, const Geometry& g, void* stream);
+int launch_rearrange(const RearrangeParams& p, bool forward, void* stream);
+int attn_smem_bytes(int d);
+
+}  // namespace skiparse

@@ -1,0 +1,139 @@
+/*
+ * skiparse.h -- C ABI of libskiparse.so: Skiparse-2D sparse attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (paper.rainbus.top summary of "OSP-Next: Efficient High-Quality Video Generation
+ * with Sparse Sequence Parallelism, HiF8 Quantization, and Reinforcement Learning", sections
+ * 核心方法 (core method) and 方法步骤详情 (method step details)):
+ *   video tokens of shape (B, T, H, W, C) with C = heads*d are split into P^2 subsequences;
+ *   token-wise mode (pixel-unshuffle-like) puts token (h, w) in class (h mod P, w mod P),
+ *   group-wise mode (patch-unshuffle-like) puts it in class ((h div P) mod P, (w div P) mod P);
+ *   when H or W is not a multiple of P^2 the grid is padded up to the next multiple and the
+ *   padded keys are masked; every subsequence runs dense softmax attention; the result is
+ *   rearranged back to the original layout.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are bfloat16, contiguous (row-major), device pointers, 16-byte aligned.
+ *   - Original layout: (B, T, H, W, heads, d). Rearranged layout: (B*P*P, n, heads, d) with
+ *     n = T * (Hp/P) * (Wp/P), Hp = ceil(H/P^2)*P^2, Wp = ceil(W/P^2)*P^2; subsequence index
+ *     b*P*P + ci*P + cj; inside a subsequence tokens are in (t, r, s) raster order, where (r, s)
+ *     is the token's position in its class's sub-grid: r = h div P (token-wise) or
+ *     (h div P^2)*P + h mod P (group-wise), and s likewise from w. Padding is at the
+ *     bottom/right of each frame.
+ *   - Softmax scale is 1/sqrt(d); no causal mask, no dropout, no bias.
+ *   - Ownership: the caller allocates and owns every buffer. The library allocates no device
+ *     memory per call; its only device state is one status word per device.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *     Argument errors are reported synchronously, before any launch, and nothing is launched.
+ *     No function throws across the ABI.
+ *   - Supported: 1 <= B, T, H, W, heads; d in {32, 64, 128}; 1 <= P <= 8;
+ *     mode in {SKIPARSE_TOKEN_WISE, SKIPARSE_GROUP_WISE}; B*T*H*W*heads < 2^31.
+ */
+#ifndef SKIPARSE_H
+#define SKIPARSE_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SKIPARSE_API __attribute__((visibility("default")))
+#else
+#define SKIPARSE_API
+#endif
+
+/* Opaque CUDA stream handle; identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* skiparse_stream_t;
+
+enum { SKIPARSE_TOKEN_WISE = 0, SKIPARSE_GROUP_WISE = 1 };
+
+enum {
+    SKIPARSE_OK = 0,
+    SKIPARSE_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad mode, aliasing */
+    SKIPARSE_ERR_UNSUPPORTED = 2, /* valid but outside the supported set (d, P, size) */
+    SKIPARSE_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+    SKIPARSE_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+    SKIPARSE_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired; its output is invalid */
+};
+
+/*
+ * Skiparse-2D attention forward, fused: the class rearrange, the pad-key mask, the dense
+ * attention of every subsequence and the inverse rearrange, in one kernel launch.
+ * (核心方法 and 方法步骤详情 on the summary page; the English abstract on chatpaper.ai.)
+ *
+ *   q, k, v : (B, T, H, W, heads, d) bf16, read-only.
+ *   out     : (B, T, H, W, heads, d) bf16, written entirely (every real token has an output).
+ *             Must not overlap q, k or v (SKIPARSE_ERR_INVALID_ARG).
+ *   For every real query token x of class c in batch b and every head:
+ *     out[x] = sum_y softmax_y(q[x].k[y] / sqrt(d)) v[y] over the real tokens y of class c,
+ *   accumulated in fp32, rounded once to bf16. P = 1 is dense full attention.
+ * Returns SKIPARSE_OK once the kernel is queued. Device-side failures (a bounded wait that
+ * expired) are reported by skiparse_get_device_status().
+ */
+SKIPARSE_API int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                        int B, int T, int H, int W, int heads, int d, int P, int mode,
+                        skiparse_stream_t stream);
+
+/*
+ * Rearrange (方法步骤详情: the rearrange that forms the P^2 subsequences, with padding).
+ *   x : (B, T, H, W, heads, d) bf16, read-only.
+ *   y : (B*P*P, n, heads, d) bf16, skiparse_rearranged_numel() elements, written entirely;
+ *       pad slots are written as +0.0. Must not overlap x.
+ * A bit-exact permutation of whole (heads*d) token rows.
+ */
+SKIPARSE_API int skiparse_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d,
+                       int P, int mode, skiparse_stream_t stream);
+
+/*
+ * Inverse rearrange (方法步骤详情: rearranged back to the original layout).
+ *   y : (B*P*P, n, heads, d) bf16, read-only; pad slots are ignored.
+ *   x : (B, T, H, W, heads, d) bf16, written entirely. Must not overlap y.
+ */
+SKIPARSE_API int skiparse_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
+                         int P, int mode, skiparse_stream_t stream);
+
+/* Number of elements of the rearranged tensor, B*P*P*n*heads*d; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse_rearranged_numel(int B, int T, int H, int W, int heads, int d, int P);
+
+/* H or W padded to the next multiple of P*P; -1 on invalid arguments. */
+SKIPARSE_API int skiparse_padded_extent(int X, int P);
+
+/* Padded subsequence length n = T*(Hp/P)*(Wp/P); -1 on invalid arguments. */
+SKIPARSE_API long long skiparse_subseq_len(int T, int H, int W, int P);
+
+/* Number of real tokens of class (ci, cj) in one batch element; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse_class_len(int T, int H, int W, int P, int mode, int ci, int cj);
+
+/*
+ * Synchronizes `stream`, then returns and clears the current device's error word: SKIPARSE_OK,
+ * or SKIPARSE_ERR_TIMEOUT if any kernel since the last call gave up on a bounded wait (its
+ * output is then invalid), or SKIPARSE_ERR_CUDA if the synchronization itself failed.
+ */
+SKIPARSE_API int skiparse_get_device_status(skiparse_stream_t stream);
+
+/* Static, human-readable name of a status code. Never NULL. */
+SKIPARSE_API const char* skiparse_status_string(int status);
+
+/* Library version string, static. */
+SKIPARSE_API const char* skiparse_version(void);
+
+/*
+ * Bound, in nanoseconds, on every wait inside a kernel (default 2e9 = 2 s). After the bound a
+ * kernel records SKIPARSE_ERR_TIMEOUT and returns instead of hanging. Applies to later
+ * launches from any thread. ns == 0 restores the default. Returns the previous value.
+ */
+SKIPARSE_API unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Test hook for failure detection. kind = 1 makes the next skiparse2d_attn_fwd launch on this
+ * host thread's process expect 16 more bytes on its first K-tile barrier than are ever
+ * delivered, so that the consumer's bounded wait expires and the kernel reports
+ * SKIPARSE_ERR_TIMEOUT without faulting or hanging the GPU. kind = 0 clears it. The hook is
+ * consumed by one launch. Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
+ */
+SKIPARSE_API int skiparse_debug_inject_fault(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKIPARSE_H */

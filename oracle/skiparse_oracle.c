@@ -298,6 +298,41 @@ int oracle_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, dou
     return rc;
 }
 
+/* The forward pass for selected output rows. The pages' three steps restricted to what
+ * those rows need: for every (subsequence, head) that holds a requested query, the rearrange
+ * of step 1 is run for that one subsequence and head (same index loops and pad mask as
+ * oracle_rearrange), step 2 attends each requested query over it, and step 3 writes the
+ * result to the requested row's slot of out_rows. */
+typedef struct {
+    const uint16_t *sq, *sk, *sv;   /* one subsequence, one head: (n, d) */
+    const uint8_t* valid;
+    long long n;
+    int d;
+    const long long* pos;           /* query positions inside the subsequence */
+    const long long* slot;          /* where each result goes in out_rows */
+    long long count;
+    double* out;
+    int tid, nthreads;
+} rows_job;
+
+static void* rows_worker(void* arg) {
+    rows_job* jb = (rows_job*)arg;
+    double* score = (double*)malloc(sizeof(double) * (size_t)jb->n);
+    if (!score) return (void*)1;
+    for (long long u = jb->tid; u < jb->count; u += jb->nthreads) {
+        /* heads = 1 view: the gathered buffers hold only this head */
+        attend_one(jb->sq, jb->sk, jb->sv, jb->valid, jb->n, 1, jb->d, 0, jb->pos[u], 0,
+                   jb->out + jb->slot[u] * (long long)jb->d, score);
+    }
+    free(score);
+    return NULL;
+}
+
+static int cmp_ll(const void* a, const void* b) {
+    const long long x = *(const long long*)a, y = *(const long long*)b;
+    return x < y ? -1 : x > y;
+}
+
 int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const long long* rows, long long nrows, double* out_rows,
                          int B, int T, int H, int W, int heads, int d, int P, int mode,
@@ -306,15 +341,15 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
     const long long ntok = (long long)B * T * H * W;
     for (long long i = 0; i < nrows; ++i)
         if (rows[i] < 0 || rows[i] >= ntok * heads) return -1;
-    rearranged r;
-    long long n = 0;
-    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
-    if (rc) return rc;
+    if (nrows == 0) return 0;
+    if (nthreads < 1) nthreads = 1;
     const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
     const int R = Hp / P, S = Wp / P;
-    long long* units = (long long*)malloc(sizeof(long long) * (size_t)(nrows > 0 ? nrows : 1));
-    if (!units) { free_rearranged(&r); return -2; }
-    /* map each requested original (token, head) to its subsequence slot */
+    const long long n = (long long)T * R * S;
+    const long long q2 = (long long)P * P;
+    /* key = ((seq*heads + head) * n + pos), packed with the request index for sorting */
+    long long* key = (long long*)malloc(sizeof(long long) * (size_t)nrows * 2);
+    if (!key) return -2;
     for (long long i = 0; i < nrows; ++i) {
         const int head = (int)(rows[i] % heads);
         long long tok = rows[i] / heads;
@@ -325,19 +360,69 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
         int ci, rr, cj, ss;
         oracle_axis_map(h, P, mode, &ci, &rr);
         oracle_axis_map(w, P, mode, &cj, &ss);
-        const long long seq = (long long)b * P * P + ci * P + cj;
+        const long long seq = (long long)b * q2 + ci * P + cj;
         const long long pos = ((long long)t * R + rr) * S + ss;
-        units[i] = (seq * n + pos) * heads + head;
+        key[2 * i] = (seq * heads + head) * n + pos;
+        key[2 * i + 1] = i;
     }
-    attn_job jb;
-    memset(&jb, 0, sizeof jb);
-    jb.yq = r.yq; jb.yk = r.yk; jb.yv = r.yv; jb.valid = r.valid;
-    jb.n = n; jb.heads = heads; jb.d = d;
-    jb.nunits = nrows;
-    jb.units = units;
-    jb.out = out_rows;
-    rc = nrows > 0 ? run_attention(jb, nthreads) : 0;
-    free(units);
-    free_rearranged(&r);
+    qsort(key, (size_t)nrows, 2 * sizeof(long long), cmp_ll);
+    uint16_t* sq = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint16_t* sk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint16_t* sv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint8_t* valid = (uint8_t*)malloc((size_t)n);
+    long long* pos = (long long*)malloc(sizeof(long long) * (size_t)nrows);
+    long long* slot = (long long*)malloc(sizeof(long long) * (size_t)nrows);
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    rows_job* jobs = (rows_job*)malloc(sizeof(rows_job) * (size_t)nthreads);
+    int rc = 0;
+    if (!sq || !sk || !sv || !valid || !pos || !slot || !th || !jobs) rc = -2;
+    for (long long g0 = 0; rc == 0 && g0 < nrows;) {
+        const long long group = key[2 * g0] / n;  /* seq*heads + head */
+        long long g1 = g0;
+        while (g1 < nrows && key[2 * g1] / n == group) {
+            pos[g1 - g0] = key[2 * g1] % n;
+            slot[g1 - g0] = key[2 * g1 + 1];
+            ++g1;
+        }
+        const long long seq = group / heads;
+        const int head = (int)(group % heads);
+        const int b = (int)(seq / q2);
+        const int c = (int)(seq % q2);
+        /* step 1 for this subsequence and head: same loops as oracle_rearrange */
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hp; ++h)
+                for (int w = 0; w < Wp; ++w) {
+                    int ci, rr, cj, ss;
+                    oracle_axis_map(h, P, mode, &ci, &rr);
+                    oracle_axis_map(w, P, mode, &cj, &ss);
+                    if (ci * P + cj != c) continue;
+                    const long long p = ((long long)t * R + rr) * S + ss;
+                    const int real = (h < H) && (w < W);
+                    valid[p] = (uint8_t)real;
+                    const long long src = ((((long long)b * T + t) * H + h) * W + w) * heads + head;
+                    for (int e = 0; e < d; ++e) {
+                        sq[p * d + e] = real ? q[src * d + e] : 0;
+                        sk[p * d + e] = real ? k[src * d + e] : 0;
+                        sv[p * d + e] = real ? v[src * d + e] : 0;
+                    }
+                }
+        /* step 2 for the requested queries, step 3 by writing to their slots */
+        int started = 0;
+        for (int t = 0; t < nthreads; ++t) {
+            rows_job* jb = &jobs[t];
+            jb->sq = sq; jb->sk = sk; jb->sv = sv; jb->valid = valid;
+            jb->n = n; jb->d = d; jb->pos = pos; jb->slot = slot; jb->count = g1 - g0;
+            jb->out = out_rows; jb->tid = t; jb->nthreads = nthreads;
+            if (pthread_create(&th[t], NULL, rows_worker, jb) != 0) { rc = -3; break; }
+            ++started;
+        }
+        for (int t = 0; t < started; ++t) {
+            void* ret = NULL;
+            pthread_join(th[t], &ret);
+            if (ret) rc = -2;
+        }
+        g0 = g1;
+    }
+    free(key); free(sq); free(sk); free(sv); free(valid); free(pos); free(slot); free(th); free(jobs);
     return rc;
 }

@@ -1,0 +1,136 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the header
+declares, computes the Skiparse geometry, and rejects bad arguments synchronously
+(before any CUDA call)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from fixed_pattern_sparse_b200 import _lib
+from fixed_pattern_sparse_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "skiparse.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^SKIPARSE_API [^(]*?\b(skiparse\w*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("skiparse2d_attn_fwd", "skiparse_rearrange", "skiparse_unrearrange",
+                 "skiparse_get_device_status", "skiparse_status_string"):
+        assert must in names
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_exports_are_only_the_c_abi():
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {n for n in exported if n.startswith("skiparse")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings(L):
+    for code, name in _lib.STATUS.items():
+        assert L.skiparse_status_string(code).decode() == name
+    assert L.skiparse_status_string(99).decode() == "SKIPARSE_ERR_UNKNOWN"
+    assert b"sm_100a" in L.skiparse_version()
+
+
+@pytest.mark.parametrize("X,P", [(45, 2), (80, 2), (48, 3), (84, 3), (1, 2), (13, 4), (7, 1), (100, 8)])
+def test_padded_extent_matches_oracle(L, X, P):
+    assert L.skiparse_padded_extent(X, P) == oracle.padded_extent(X, P)
+
+
+def test_geometry_matches_oracle(L):
+    """Real per-class token counts of the product's geometry against the oracle's rearrange."""
+    import numpy as np
+    for (T, H, W, P) in [(2, 8, 8, 2), (3, 10, 14, 2), (1, 5, 7, 3), (2, 3, 20, 4), (1, 45, 80, 2),
+                         (1, 48, 84, 3), (2, 6, 5, 1)]:
+        assert L.skiparse_subseq_len(T, H, W, P) == oracle.subseq_len(T, H, W, P)
+        for mode in (0, 1):
+            x = (np.arange(T * H * W, dtype=np.uint16) + 1).reshape(1, T, H, W, 1, 1)
+            y = oracle.rearrange(x, P, mode)
+            for ci in range(P):
+                for cj in range(P):
+                    real = int((y[ci * P + cj, :, 0, 0] > 0).sum())
+                    assert L.skiparse_class_len(T, H, W, P, mode, ci, cj) == real
+        n = L.skiparse_rearranged_numel(2, T, H, W, 3, 64, P)
+        assert n == 2 * P * P * oracle.subseq_len(T, H, W, P) * 3 * 64
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails before any CUDA call
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, FAKE, FAKE, FAKE + 4096, 1, 2, 8, 8, 2, 32, 2, 0), 1),          # null q
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 48, 2, 0), 2),   # d = 48 unsupported
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 32, 9, 0), 2),   # P = 9 unsupported
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 32, 2, 2), 1),   # bad mode
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 20), 0, 2, 8, 8, 2, 32, 2, 0), 1),   # B = 0
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, -8, 8, 2, 32, 2, 0), 1),  # negative H
+    ((FAKE + 8, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 32, 2, 0), 3),  # misaligned q
+    ((FAKE, FAKE, FAKE, FAKE + 2, 1, 2, 8, 8, 2, 32, 2, 0), 3),           # misaligned out
+    ((FAKE, FAKE + (1 << 20), FAKE + (2 << 20), FAKE, 1, 2, 8, 8, 2, 32, 2, 0), 1),  # out aliases q
+    ((FAKE, FAKE, FAKE, FAKE + 4096, 1, 2, 8, 8, 2, 32, 2, 0), 1),        # out overlaps q's range
+    ((FAKE, FAKE, FAKE, FAKE + (1 << 30), 64, 21, 480, 840, 40, 128, 2, 0), 2),  # > 2^31 rows
+])
+def test_attn_fwd_rejects_bad_arguments_synchronously(L, args, code):
+    assert L.skiparse2d_attn_fwd(*args, None) == code
+
+
+def test_rearrange_rejects_bad_arguments_synchronously(L):
+    assert L.skiparse_rearrange(0, FAKE, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
+    assert L.skiparse_rearrange(FAKE, FAKE + 4, 1, 2, 8, 8, 2, 32, 2, 0, None) == 3
+    assert L.skiparse_rearrange(FAKE, FAKE, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1  # in place
+    assert L.skiparse_unrearrange(FAKE, FAKE + 64, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1  # overlap
+    assert L.skiparse_unrearrange(FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 40, 2, 0, None) == 2
+
+
+def test_wait_limit_and_fault_hook(L):
+    prev = L.skiparse_set_wait_limit_ns(123456)
+    assert prev == 2_000_000_000
+    assert L.skiparse_set_wait_limit_ns(0) == 123456
+    assert L.skiparse_set_wait_limit_ns(0) == 2_000_000_000
+    assert L.skiparse_debug_inject_fault(2) == 1
+    assert L.skiparse_debug_inject_fault(0) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import fixed_pattern_sparse_b200 as fps
+    x = torch.zeros((1, 1, 4, 4, 1, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fps.skiparse2d_attn_fwd(x, x, x, 2, 0)
+    with pytest.raises(ValueError):
+        fps.skiparse_rearrange(x, 2, 0)
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "fixed_pattern_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower().replace("oracles", ""), f

@@ -1,0 +1,47 @@
+"""Failure detection without a GPU fault: every wait in the attention kernel is bounded.
+
+The test hook makes one launch expect 16 more bytes on its first K-tile barrier than the
+TMA ever delivers, so the MMA warp's wait runs out (a flag that nothing sets). The kernel
+must then record SKIPARSE_ERR_TIMEOUT in the device status word, release its tensor
+memory and return; the context stays usable and the next launch is correct."""
+
+from __future__ import annotations
+
+import time
+
+import pytest
+import torch
+
+import oracle
+import skiparse_synth as synth
+from parity_helpers import check_close
+
+pytestmark = pytest.mark.gpu
+
+
+def test_lost_arrival_times_out_and_recovers():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import fixed_pattern_sparse_b200 as fps
+    from fixed_pattern_sparse_b200 import _lib
+    L = _lib.lib()
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.qkv(w)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    assert fps.get_device_status() == 0
+    prev = L.skiparse_set_wait_limit_ns(100_000_000)  # 0.1 s
+    try:
+        assert L.skiparse_debug_inject_fault(1) == 0
+        t0 = time.time()
+        fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, 0)
+        status = fps.get_device_status()
+        elapsed = time.time() - t0
+        assert status == 5, f"expected SKIPARSE_ERR_TIMEOUT, got {status}"
+        assert elapsed < 30
+    finally:
+        L.skiparse_debug_inject_fault(0)
+        L.skiparse_set_wait_limit_ns(prev)
+    # the context is still usable and the next launch is right
+    out = fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, 0)
+    assert fps.get_device_status() == 0
+    check_close(out.to(torch.float64).cpu().numpy(), oracle.attn_fwd(q, k, v, w.P, 0), "after timeout")
