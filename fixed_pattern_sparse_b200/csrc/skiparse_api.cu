@@ -1,13 +1,11 @@
 // skiparse_api.cu -- the C ABI of libskiparse.so (declared in include/skiparse.h):
-// argument validation, Skiparse-2D geometry, TMA tensor-map encoding, kernel launch and the
-// per-device status word. Nothing here allocates device memory.
-#include <cuda.h>
+// argument validation, Skiparse-2D geometry, kernel launch and the per-device status word.
+// Nothing here allocates device memory.
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "../../include/skiparse.h"
 #include "skiparse_internal.cuh"
@@ -22,25 +20,6 @@ std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_fault{0};
 
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
 
 int padded(int X, int P) { return ((X + P * P - 1) / (P * P)) * (P * P); }
 
@@ -90,23 +69,6 @@ int* status_ptr() {
         return nullptr;
     }
     return p;
-}
-
-// 2-D view (rows = tokens*heads, cols = d) of a (…, heads, d) bf16 tensor, box = one row x
-// (64 or 32) columns, swizzled so the tile lands in the UMMA canonical K-major layout.
-int encode_rows_map(CUtensorMap* map, const void* base, long long rows, int d) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return SKIPARSE_ERR_CUDA;
-    const int box_cols = d >= 64 ? 64 : 32;
-    const CUtensorMapSwizzle sw = d >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
 }
 
 }  // namespace
@@ -191,11 +153,10 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     const size_t bytes = static_cast<size_t>(rows) * d * 2;
     if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
         return SKIPARSE_ERR_INVALID_ARG;
-    alignas(64) CUtensorMap tq, tk, tv;
-    if (encode_rows_map(&tq, q, rows, d) || encode_rows_map(&tk, k, rows, d) ||
-        encode_rows_map(&tv, v, rows, d))
-        return SKIPARSE_ERR_CUDA;
     skiparse::AttnParams p{};
+    p.q = static_cast<const uint16_t*>(q);
+    p.k = static_cast<const uint16_t*>(k);
+    p.v = static_cast<const uint16_t*>(v);
     p.out = static_cast<uint16_t*>(out);
     p.status = status_ptr();
     if (!p.status) return SKIPARSE_ERR_CUDA;
@@ -207,7 +168,7 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.exchange(0);
-    const int e = skiparse::launch_attn_fwd(&tq, &tk, &tv, p, g, stream);
+    const int e = skiparse::launch_attn_fwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
 }
 

@@ -45,15 +45,18 @@ struct Geometry {
     int Sc[kMaxP];     // real sub-grid columns of class column cj
 };
 
-// Parameters of the fused attention kernel (plain values only; tensor maps are separate).
+// Parameters of the fused attention kernel.
 struct AttnParams {
-    uint16_t* out;                 // bf16 bits, (B,T,H,W,heads,d)
+    const uint16_t* q;             // bf16 bits, (B,T,H,W,heads,d)
+    const uint16_t* k;
+    const uint16_t* v;
+    uint16_t* out;
     int* status;                   // device error word
     int T, H, W, heads, P, mode;
     int Rc[kMaxP], Sc[kMaxP];
     float scale_log2;              // log2(e)/sqrt(d)
     unsigned long long wait_limit_ns;
-    int fault;                     // test hook: 1 = under-deliver the first K tile
+    int fault;                     // test hook: 1 = one producer never signals the first K tile
 };
 
 struct RearrangeParams {
@@ -69,8 +72,7 @@ struct RearrangeParams {
 enum : int { kOk = 0, kErrTimeout = 5 };
 
 // Launchers (defined in the kernel translation units). They return the cudaError_t as int.
-int launch_attn_fwd(const void* tmap_q, const void* tmap_k, const void* tmap_v,
-                    const AttnParams& p, const Geometry& g, void* stream);
+int launch_attn_fwd(const AttnParams& p, const Geometry& g, void* stream);
 int launch_rearrange(const RearrangeParams& p, bool forward, void* stream);
 int attn_smem_bytes(int d);
 

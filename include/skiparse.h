@@ -124,11 +124,11 @@ SKIPARSE_API const char* skiparse_version(void);
 SKIPARSE_API unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns);
 
 /*
- * Test hook for failure detection. kind = 1 makes the next skiparse2d_attn_fwd launch on this
- * host thread's process expect 16 more bytes on its first K-tile barrier than are ever
- * delivered, so that the consumer's bounded wait expires and the kernel reports
- * SKIPARSE_ERR_TIMEOUT without faulting or hanging the GPU. kind = 0 clears it. The hook is
- * consumed by one launch. Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
+ * Test hook for failure detection. kind = 1 makes the next skiparse2d_attn_fwd launch of this
+ * process lose one arrival on its first K-tile barrier (one producer thread never signals it),
+ * so that the consumer's bounded wait expires and the kernel reports SKIPARSE_ERR_TIMEOUT
+ * without faulting or hanging the GPU. kind = 0 clears it. The hook is consumed by one launch.
+ * Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
  */
 SKIPARSE_API int skiparse_debug_inject_fault(int kind);
 
