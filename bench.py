@@ -44,7 +44,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the attention kernel, from an ncu capture, keyed by the hash of
 # the kernel sources it was captured on (a changed kernel reports null until re-captured).
-KNOWN_TRAFFIC = {}
+KNOWN_TRAFFIC = {
+    # 480p capture (dram__bytes_read.sum + dram__bytes_write.sum = 384.1 MB per launch), scaled to
+    # the 720p launch by the ratio of token rows (7.692); traffic grows with q/k/v/out because the
+    # kernel reads each input once and writes the output once.
+    "2a906497c379c4ad": 2.955e9,
+}
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
                 "fixed_pattern_sparse_b200/csrc/ptx_sm100.cuh",
@@ -275,7 +280,7 @@ def run_ours(args):
     ms_step = total_ms / args.steps
     value = fl * args.steps * world / (total_ms / 1e3) / 1e12
     by_mode = {MODE_NAME[m]: statistics.mean(per_launch[i] for i in range(args.steps) if i % len(modes) == j)
-               for j, m in enumerate(modes)}
+               for j, m in enumerate(modes) if j < args.steps}
 
     peaks, peak_src = load_peaks()
     mean_launch_s = statistics.mean(per_launch) / 1e3
@@ -328,6 +333,36 @@ def run_ours(args):
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the dense comparison")
 
+    # standalone rearrange / unrearrange bandwidth (HBM-bound permutation of token rows)
+    rearr = None
+    if not args.no_rearrange:
+        yshape = fps.rearranged_shape(q.shape, w.P)
+        y = torch.empty(yshape, dtype=torch.bfloat16, device=dev)
+        back = torch.empty_like(qd)
+        bytes_fwd = (qd.numel() + y.numel()) * 2  # read real rows, write all slots
+        bytes_inv = 2 * qd.numel() * 2            # read real slots, write all rows
+        res = {}
+        for name, fn, nbytes in (("rearrange", lambda m: fps.skiparse_rearrange(qd, w.P, m, out=y), bytes_fwd),
+                                 ("unrearrange", lambda m: fps.skiparse_unrearrange(y, q.shape, w.P, m, out=back), bytes_inv)):
+            for i in range(3):
+                fn(modes[i % len(modes)])
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            for i in range(args.rearrange_steps):
+                fn(modes[i % len(modes)])
+            r1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = r0.elapsed_time(r1) / args.rearrange_steps
+            gbs = nbytes / (ms / 1e3) / 1e9
+            res[name] = {"ms": round(ms, 4), "bytes": nbytes, "gbs": round(gbs, 1),
+                         "frac_of_hbm": round(gbs / float(peaks["hbm_gbs"]), 4)}
+        res["hbm_peak_gbs"] = float(peaks["hbm_gbs"])
+        res["note"] = "algorithmic bytes (read + write) per call / CUDA-event time; inputs > L2"
+        rearr = res
+        del y, back
+        if fps.get_device_status() != 0:
+            raise SystemExit("device status error in the rearrange timing")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -337,7 +372,8 @@ def run_ours(args):
                "sample": desc, "seconds": round(dt, 2)}
 
     if rank == 0:
-        real = {MODE_NAME[m]: round(flops_real(w, m) / (by_mode[MODE_NAME[m]] / 1e3) / 1e12, 1) for m in modes}
+        real = {MODE_NAME[m]: round(flops_real(w, m) / (by_mode[MODE_NAME[m]] / 1e3) / 1e12, 1)
+                for m in modes if MODE_NAME[m] in by_mode}
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
@@ -356,6 +392,7 @@ def run_ours(args):
             "ms_per_layer": {k_: round(v_, 3) for k_, v_ in by_mode.items()},
             "tflops_real_pairs": real,
             "dense_p1": dense,
+            "rearrange_kernels": rearr,
             "kernel_hash": kernel_hash(),
         }
         print(json.dumps(line), flush=True)
@@ -428,6 +465,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rearrange", action="store_true")
+    ap.add_argument("--rearrange-steps", type=int, default=10)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

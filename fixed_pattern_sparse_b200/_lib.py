@@ -25,8 +25,10 @@ SIGNATURES = {
     "skiparse_get_device_status": (_I, [_VP]),
     "skiparse_status_string": (_CP, [_I]),
     "skiparse_version": (_CP, []),
+    "skiparse_last_error_string": (_CP, []),
     "skiparse_set_wait_limit_ns": (_ULL, [_ULL]),
     "skiparse_debug_inject_fault": (_I, [_I]),
+    "skiparse_debug_exp2": (_I, [_VP, _VP, _LL, _I, _VP]),
 }
 
 STATUS = {0: "SKIPARSE_OK", 1: "SKIPARSE_ERR_INVALID_ARG", 2: "SKIPARSE_ERR_UNSUPPORTED",
@@ -60,4 +62,7 @@ def lib() -> ctypes.CDLL:
 
 def check(code: int, what: str) -> None:
     if code != 0:
-        raise SkiparseError(code, what)
+        err = SkiparseError(code, what)
+        if code == 4:  # SKIPARSE_ERR_CUDA: add the CUDA message
+            err.args = (f"{err.args[0]} ({lib().skiparse_last_error_string().decode()})",)
+        raise err

@@ -21,6 +21,9 @@
 // so the softmax of one query tile overlaps the tensor-core work of the other.
 // Softmax rescales O lazily: only when a row maximum grows by more than 2^8 (FlashAttention-4's
 // lazy rescaling); the stale maximum keeps every p <= 256, exact after the final division.
+// Options (compile-time, off by default because they measured no faster on B200): MUFU turns
+// between the two softmax warpgroups, exponentials against a stale running max, part of the
+// exponentials as a polynomial on the FMA pipe (a FlashAttention-4 idea), a setmaxnreg split.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -32,11 +35,34 @@ namespace {
 
 constexpr int kBM = 128;   // queries per tile == TMEM lanes
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 352;
+// Register split: 12 warps; the softmax warpgroups raise their register budget with
+// setmaxnreg while the producer/MMA warpgroup lowers its own.
+#ifndef SKIPARSE_REGSPLIT
+#define SKIPARSE_REGSPLIT 0
+#endif
+// Optional softmax schedules, measured no faster on B200 and therefore off by default:
+// MUFU turns (the two softmax warpgroups take turns on the exponential unit) and stale-max
+// exponentials (taken against the running max while the next chunk of S loads).
+#ifndef SKIPARSE_MUFU_TURNS
+#define SKIPARSE_MUFU_TURNS 0
+#endif
+#ifndef SKIPARSE_STALE_MAX
+#define SKIPARSE_STALE_MAX 0
+#endif
+constexpr int kThreads = SKIPARSE_REGSPLIT ? 384 : 352;
+constexpr int kLaunchRegs = 168;       // 65536 / 384 rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 216;      // 2 x 128 x 216 + 128 x 64 <= 384 x 168
+constexpr int kOtherRegs = 64;
 constexpr int kProdWarp0 = 8;
 constexpr int kNumProducers = 64;
 constexpr int kMmaWarp = 10;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+// Which of the 16 column pairs of every 32-column chunk take exp2 on the FMA pipe (polynomial)
+// instead of the MUFU unit. 0: none (fastest measured: MUFU is not this kernel's limiter).
+#ifndef SKIPARSE_EMU_MASK
+#define SKIPARSE_EMU_MASK 0x0000u
+#endif
+constexpr unsigned kEmuMask = SKIPARSE_EMU_MASK;
 
 template <int D>
 struct Cfg {
@@ -62,7 +88,8 @@ struct Cfg {
     static constexpr int B_VEMPTY = B_VFULL + VST;
     static constexpr int B_SFULL = B_VEMPTY + VST;        // 2: one per query tile
     static constexpr int B_PFULL = B_SFULL + 2;           // 2
-    static constexpr int B_OFULL = B_PFULL + 2;
+    static constexpr int B_TURN = B_PFULL + 2;            // 2: MUFU turn of query tile 0 / 1
+    static constexpr int B_OFULL = B_TURN + 2;
     static constexpr int B_DRAIN = B_OFULL + 1;
     static constexpr int NBARS = B_DRAIN + 1;
     static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
@@ -138,6 +165,46 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restri
     }
 }
 
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t* v) {
+    float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
+    float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
+#pragma unroll
+    for (int e = 4; e < N; e += 4) {
+        m0 = fmaxf(m0, __uint_as_float(v[e]));
+        m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+        m2 = fmaxf(m2, __uint_as_float(v[e + 2]));
+        m3 = fmaxf(m3, __uint_as_float(v[e + 3]));
+    }
+    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// p = 2^(s*sl2 + neg) for 32 scores; the bf16 pairs go to 16 TMEM columns at p_addr (over the
+// scores already read). EMU selects the column pairs of kEmuMask for the FMA-pipe polynomial.
+// Returns the fp32 sum of the 32 probabilities.
+template <bool EMU>
+__device__ __forceinline__ float exp_chunk(const uint32_t* v, float sl2, float neg, uint32_t p_addr) {
+    uint32_t pk[16];
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float x0 = fmaf(__uint_as_float(v[2 * e]), sl2, neg);
+        const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sl2, neg);
+        float p0, p1;
+        if (EMU && (kEmuMask & (1u << e))) {
+            ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), p0, p1);
+        } else {
+            p0 = ptx::ex2_approx(x0);
+            p1 = ptx::ex2_approx(x1);
+        }
+        s0 += p0;
+        s1 += p1;
+        pk[e] = ptx::pack_bf16x2(p0, p1);
+    }
+    ptx::tmem_st16(p_addr, pk);
+    return s0 + s1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const AttnParams p) {
     using C = Cfg<D>;
@@ -179,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
             ptx::mbar_init(bar(C::B_PFULL + i), kBM);
+            ptx::mbar_init(bar(C::B_TURN + i), kBM);
         }
         ptx::mbar_init(bar(C::B_OFULL), 1);
         ptx::mbar_init(bar(C::B_DRAIN), 1);
@@ -194,7 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProdWarp0 || warp == kProdWarp0 + 1) {
+    if (warp >= kProdWarp0) {
+#if SKIPARSE_REGSPLIT
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+#endif
+      if (warp == kProdWarp0 || warp == kProdWarp0 + 1) {
         // ------------------------------------------------------------------ producers
         // Load order Q, K0, V0, K1, V1, ... Each load is one cp.async group; a load's full
         // barrier is signalled (after this thread's copies completed and a proxy fence) once
@@ -242,53 +314,54 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             const uint32_t idesc_s = ptx::idesc_bf16_f32(kBM, kBN, false);
             const uint32_t idesc_o = ptx::idesc_bf16_f32(kBM, D, true);
             const uint32_t q0 = sbase + C::OFF_Q, q1 = q0 + C::TILE_BYTES;
-            auto issue_s = [&](uint32_t qs, uint32_t ks, uint32_t d_tmem) {
+            // Descriptors are built once; a K-step only advances the 14-bit start-address field.
+            const uint64_t qd0 = ptx::smem_desc(q0, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t qd1 = ptx::smem_desc(q1, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t kd0 = ptx::smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t vd0 = ptx::smem_desc(sbase + C::OFF_V, C::BOX_BYTES, 8 * C::SW, C::LAYOUT);
+            auto issue_s = [&](uint64_t qd, int kslot, uint32_t d_tmem) {
+                const uint64_t kd = kd0 + ((kslot * C::TILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::KSTEPS; ++kk) {
-                    const uint32_t off = (kk / C::KPB) * C::BOX_BYTES + (kk % C::KPB) * 32;
-                    const uint64_t ad = ptx::smem_desc(qs + off, 16, 8 * C::SW, C::LAYOUT);
-                    const uint64_t bd = ptx::smem_desc(ks + off, 16, 8 * C::SW, C::LAYOUT);
-                    ptx::mma_ss(d_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk / C::KPB) * C::BOX_BYTES + (kk % C::KPB) * 32) >> 4;
+                    ptx::mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_o = [&](uint32_t p_tmem, uint32_t vs, uint32_t d_tmem, bool acc) {
+            auto issue_o = [&](uint32_t p_tmem, int vslot, uint32_t d_tmem, bool acc) {
+                const uint64_t vd = vd0 + ((vslot * C::TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t bd = ptx::smem_desc(vs + kk * 16 * C::SW, C::BOX_BYTES, 8 * C::SW, C::LAYOUT);
-                    ptx::mma_ts(d_tmem, p_tmem + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    ptx::mma_ts(d_tmem, p_tmem + kk * 8, vd + ((kk * 16 * C::SW) >> 4), idesc_o,
+                                (acc || kk > 0) ? 1u : 0u);
             };
             bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort, lim) &&
                       ptx::mbar_wait(bar(C::B_KFULL + 0), 0, abort, lim);
             if (ok) {
                 ptx::tc_fence_after();
-                const uint32_t k0 = sbase + C::OFF_K;
-                issue_s(q0, k0, tmem + C::COL_S0);
+                issue_s(qd0, 0, tmem + C::COL_S0);
                 ptx::mma_commit(bar(C::B_SFULL + 0));
-                issue_s(q1, k0, tmem + C::COL_S1);
+                issue_s(qd1, 0, tmem + C::COL_S1);
                 ptx::mma_commit(bar(C::B_SFULL + 1));
                 ptx::mma_commit(bar(C::B_KEMPTY + 0));
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const int vs = j % C::VST;
-                const uint32_t v_smem = sbase + C::OFF_V + vs * C::TILE_BYTES;
                 if (!ptx::mbar_wait(bar(C::B_VFULL + vs), (j / C::VST) & 1, abort, lim) ||
                     !ptx::mbar_wait(bar(C::B_PFULL + 0), j & 1, abort, lim)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                issue_o(tmem + C::COL_S0, v_smem, tmem + C::COL_O0, j > 0);
+                issue_o(tmem + C::COL_S0, vs, tmem + C::COL_O0, j > 0);
                 const bool more = j + 1 < nkv;
                 const int ks = (j + 1) % C::KST;
-                const uint32_t k_smem = sbase + C::OFF_K + ks * C::TILE_BYTES;
                 if (more) {
                     if (!ptx::mbar_wait(bar(C::B_KFULL + ks), ((j + 1) / C::KST) & 1, abort, lim)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    issue_s(q0, k_smem, tmem + C::COL_S0);
+                    issue_s(qd0, ks, tmem + C::COL_S0);
                     ptx::mma_commit(bar(C::B_SFULL + 0));
                 }
                 if (!ptx::mbar_wait(bar(C::B_PFULL + 1), j & 1, abort, lim)) {
@@ -296,10 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     break;
                 }
                 ptx::tc_fence_after();
-                issue_o(tmem + C::COL_S1, v_smem, tmem + C::COL_O1, j > 0);
+                issue_o(tmem + C::COL_S1, vs, tmem + C::COL_O1, j > 0);
                 ptx::mma_commit(bar(C::B_VEMPTY + vs));
                 if (more) {
-                    issue_s(q1, k_smem, tmem + C::COL_S1);
+                    issue_s(qd1, ks, tmem + C::COL_S1);
                     ptx::mma_commit(bar(C::B_SFULL + 1));
                     ptx::mma_commit(bar(C::B_KEMPTY + ks));
                 }
@@ -315,74 +388,130 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             ptx::mbar_wait(bar(C::B_DRAIN), 0, &never, lim);
         }
         __syncwarp();
+      }  // warp 11 (register-split layout only) has no role
     } else {
+#if SKIPARSE_REGSPLIT
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+#endif
         // ------------------------------------------------------------------ softmax (WG 0/1)
         const int qt = warp >> 2;                       // query tile 0 or 1
         const int row = threadIdx.x & 127;              // TMEM lane == row in the tile
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t s_col = qt ? C::COL_S1 : C::COL_S0;
+        const uint32_t s_addr = tmem + lane_base + (qt ? C::COL_S1 : C::COL_S0);
         const uint32_t o_col = qt ? C::COL_O1 : C::COL_O0;
         const uint32_t sfull = bar(C::B_SFULL + qt), pfull = bar(C::B_PFULL + qt);
+        // The two query tiles take turns on the MUFU unit (their exponential phases would
+        // otherwise overlap and each would run at half rate).
+        const uint32_t my_turn = bar(C::B_TURN + qt), other_turn = bar(C::B_TURN + (qt ^ 1));
         const float sl2 = p.scale_log2;
         const float thresh = kRescaleLog2 / sl2;       // in raw score units
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        if (SKIPARSE_MUFU_TURNS && qt == 1) ptx::mbar_arrive(bar(C::B_TURN + 0));  // tile 0 goes first
         for (int j = 0; j < nkv; ++j) {
             if (!ptx::mbar_wait(sfull, j & 1, abort, lim)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            float sc[kBN];
-            {
-                uint32_t sv[32];
+            const bool last = (j == nkv - 1);
+            uint32_t sv[kBN];
+            float sum = 0.f, alpha = 1.f;
+            if (!SKIPARSE_STALE_MAX || j == 0 || last) {
+                // The row max is taken over the whole tile before any exponential (the first
+                // tile sets the reference max; the ragged last tile has masked keys).
+                float sc[kBN];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    ptx::tmem_ld32(tmem + lane_base + s_col + 32 * g, sv);
+                    ptx::tmem_ld32(s_addr + 32 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * g]));
                     ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sc[32 * g + e] = __uint_as_float(sv[e]);
+                    for (int e = 0; e < 32; ++e) sc[32 * g + e] = __uint_as_float(sv[32 * g + e]);
+                }
+                if (last) {
+                    const int valid = n_c - j * kBN;
+#pragma unroll
+                    for (int e = 0; e < kBN; ++e)
+                        if (e >= valid) sc[e] = -INFINITY;
+                }
+                float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
+#pragma unroll
+                for (int e = 4; e < kBN; e += 4) {
+                    mx0 = fmaxf(mx0, sc[e]);
+                    mx1 = fmaxf(mx1, sc[e + 1]);
+                    mx2 = fmaxf(mx2, sc[e + 2]);
+                    mx3 = fmaxf(mx3, sc[e + 3]);
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                if (j == 0 || mx > m_run + thresh) {
+                    alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
+                    m_run = mx;
+                }
+                if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
+                    ok = false;
+                    break;
+                }
+                const float neg = -m_run * sl2;
+                float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float x0 = fmaf(sc[32 * g + 2 * e], sl2, neg);
+                        const float x1 = fmaf(sc[32 * g + 2 * e + 1], sl2, neg);
+                        float p0, p1;
+                        if (kEmuMask != 0u && !last && (kEmuMask & (1u << e))) {
+                            ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), p0, p1);
+                        } else {
+                            p0 = ptx::ex2_approx(x0);
+                            p1 = ptx::ex2_approx(x1);
+                        }
+                        sum0 += p0;
+                        sum1 += p1;
+                        pk[e] = ptx::pack_bf16x2(p0, p1);
+                    }
+                    ptx::tmem_st16(s_addr + 16 * g, pk);
+                }
+                sum = sum0 + sum1;
+                if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
+            } else {
+                // Steady state: exponentials against the running max while the next 32-column
+                // chunk of S is loading; the tile's max is only checked afterwards.
+                if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
+                    ok = false;
+                    break;
+                }
+                const float neg = -m_run * sl2;
+                float mx = -INFINITY;
+                ptx::tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    if (g < 3)
+                        ptx::tmem_ld32(s_addr + 32 * (g + 1), *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * (g + 1)]));
+                    mx = fmaxf(mx, row_max<32>(&sv[32 * g]));
+                    sum += exp_chunk<true>(&sv[32 * g], sl2, neg, s_addr + 16 * g);
+                    if (g < 3) ptx::tmem_wait_ld();
+                }
+                if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
+                const bool grow = mx > m_run + thresh;
+                if (__any_sync(0xffffffffu, grow)) {
+                    // Rare: this tile raised a row max by more than 2^8. Redo its P against the
+                    // new max (S is still in registers) and rescale O below.
+                    if (grow) {
+                        alpha = ptx::ex2_approx((m_run - mx) * sl2);
+                        m_run = mx;
+                    }
+                    const float neg2 = -m_run * sl2;
+                    ptx::tmem_wait_st();  // the first pass's stores land before they are redone
+                    sum = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) sum += exp_chunk<false>(&sv[32 * g], sl2, neg2, s_addr + 16 * g);
                 }
             }
-            if (j == nkv - 1) {
-                const int valid = n_c - j * kBN;
-#pragma unroll
-                for (int e = 0; e < kBN; ++e)
-                    if (e >= valid) sc[e] = -INFINITY;
-            }
-            float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
-#pragma unroll
-            for (int e = 4; e < kBN; e += 4) {
-                mx0 = fmaxf(mx0, sc[e]);
-                mx1 = fmaxf(mx1, sc[e + 1]);
-                mx2 = fmaxf(mx2, sc[e + 2]);
-                mx3 = fmaxf(mx3, sc[e + 3]);
-            }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            // lazy rescale: keep the running max unless this tile exceeds it by > 2^8
-            const bool grow = (j == 0) || (mx > m_run + thresh);
-            float alpha = 1.f;
-            if (grow) {
-                alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
-                m_run = mx;
-            }
-            const float neg = -m_run * sl2;
-            float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ptx::ex2_approx(fmaf(sc[32 * g + 2 * e], sl2, neg));
-                    const float p1 = ptx::ex2_approx(fmaf(sc[32 * g + 2 * e + 1], sl2, neg));
-                    sum0 += p0;
-                    sum1 += p1;
-                    pk[e] = ptx::pack_bf16x2(p0, p1);
-                }
-                ptx::tmem_st16(tmem + lane_base + s_col + 16 * g, pk);
-            }
-            l_run = l_run * alpha + (sum0 + sum1);
-            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+            l_run = l_run * alpha + sum;
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // O_qt was completed by the previous P*V (the commit behind this tile's S covers it)
 #pragma unroll
                 for (int g = 0; g < D / 32; ++g) {
@@ -446,6 +575,14 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
         e = cudaFuncSetAttribute(skiparse_attn_fwd_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return static_cast<int>(e);
+        if (SKIPARSE_REGSPLIT) {
+            // setmaxnreg.inc waits for registers that the block released; the split above is
+            // only safe if the block is launched with exactly kLaunchRegs per thread.
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, skiparse_attn_fwd_kernel<D>);
+            if (e != cudaSuccess) return static_cast<int>(e);
+            if (fa.numRegs != kLaunchRegs) return static_cast<int>(cudaErrorInvalidConfiguration);
+        }
         attr_done_dev[dev] = 1;
     }
     int n_max = 0;
@@ -459,7 +596,34 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
     return static_cast<int>(cudaGetLastError());
 }
 
+// Diagnostic: y = 2^x by the MUFU instruction (method 0) or the FMA-pipe polynomial (method 1)
+// exactly as the softmax evaluates them, so their error can be tested against fp64.
+__global__ void skiparse_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n,
+                                     int method) {
+    const long long i = 2 * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+    float y0, y1;
+    if (method == 1) {
+        ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), y0, y1);
+    } else {
+        y0 = ptx::ex2_approx(x0);
+        y1 = ptx::ex2_approx(x1);
+    }
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
+
+int launch_exp2(const float* x, float* y, long long n, int method, void* stream) {
+    if (n <= 0) return static_cast<int>(cudaSuccess);
+    const long long pairs = (n + 1) / 2;
+    const int threads = 256;
+    const long long blocks = (pairs + threads - 1) / threads;
+    skiparse_exp2_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, method);
+    return static_cast<int>(cudaGetLastError());
+}
 
 int attn_smem_bytes(int d) {
     switch (d) {

@@ -47,8 +47,22 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// A thread that finds the phase incomplete may be suspended (not spinning) until the phase
+// completes or about `SKIPARSE_WAIT_HINT_NS` nanoseconds pass (0: the hardware default).
+#ifndef SKIPARSE_WAIT_HINT_NS
+#define SKIPARSE_WAIT_HINT_NS 0
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
+#if SKIPARSE_WAIT_HINT_NS > 0
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(static_cast<uint32_t>(SKIPARSE_WAIT_HINT_NS))
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -56,17 +70,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
 // Waits for the phase with the given parity to complete. Bounded: gives up (returns false)
 // when *abort becomes non-zero or after limit_ns nanoseconds, so that a lost arrival can
 // never hang the GPU.
+// A waiting warp backs off with nanosleep so that it does not take issue slots from the warps
+// doing the work on the same SM sub-partition (0 disables the back-off).
+#ifndef SKIPARSE_WAIT_SLEEP_NS
+#define SKIPARSE_WAIT_SLEEP_NS 0
+#endif
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
+        if (SKIPARSE_WAIT_SLEEP_NS > 0) __nanosleep(SKIPARSE_WAIT_SLEEP_NS);
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0u) {
             if (*abort) return false;
@@ -231,6 +252,58 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---------------------------------------------------------------- packed fp32 (sm_100)
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe instead of the MUFU unit: x = n + f with n the
+// nearest integer (added to the exponent field) and f in [-1/2, 1/2], where 2^f is a degree-3
+// polynomial. Its coefficients were fitted here with the Remez exchange algorithm (minimax
+// relative error) and give max relative error 7.5e-5 in fp32 Horner form, 26x below half an
+// ulp of bf16, the precision P is kept in. x is clamped at -125 so the exponent field cannot
+// underflow (2^-125 ~ 2.4e-38 stands in for smaller results).
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);     // 1.5 * 2^23
+    const uint64_t t = f2_add(f2_pack(x0, x1), magic);           // round(x) in the low bits
+    const uint64_t nf = f2_add(t, f2_pack(-12582912.f, -12582912.f));
+    const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), f2_pack(x0, x1));
+    uint64_t p = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.242611125f, 0.242611125f));
+    p = f2_fma(p, f, f2_pack(0.693260968f, 0.693260968f));
+    p = f2_fma(p, f, f2_pack(0.999928057f, 0.999928057f));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);  // n << 23 added
+    const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
+    return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -17,6 +17,13 @@ using skiparse::Geometry;
 __device__ int g_skiparse_status = 0;  // one error word per device
 
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+thread_local const char* t_last_cuda_error = "no error";
+
+// Records a failed CUDA call's message for skiparse_last_error_string(); returns the status.
+int cuda_fail(int err) {
+    t_last_cuda_error = cudaGetErrorString(static_cast<cudaError_t>(err));
+    return SKIPARSE_ERR_CUDA;
+}
 std::atomic<int> g_fault{0};
 
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
@@ -64,8 +71,10 @@ bool overlaps(const void* a, size_t abytes, const void* b, size_t bbytes) {
 
 int* status_ptr() {
     int* p = nullptr;
-    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_skiparse_status) != cudaSuccess) {
+    const cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_skiparse_status);
+    if (e != cudaSuccess) {
         cudaGetLastError();
+        cuda_fail(e);
         return nullptr;
     }
     return p;
@@ -88,6 +97,8 @@ const char* skiparse_status_string(int status) {
 }
 
 const char* skiparse_version(void) { return "skiparse-b200 0.1 (sm_100a, tcgen05)"; }
+
+const char* skiparse_last_error_string(void) { return t_last_cuda_error; }
 
 int skiparse_padded_extent(int X, int P) {
     if (X < 1 || P < 1 || P > skiparse::kMaxP) return -1;
@@ -122,21 +133,32 @@ int skiparse_debug_inject_fault(int kind) {
     return SKIPARSE_OK;
 }
 
+int skiparse_debug_exp2(const float* x, float* y, long long n, int method,
+                        skiparse_stream_t stream) {
+    if (n < 0 || (n > 0 && (!x || !y)) || (method != 0 && method != 1)) return SKIPARSE_ERR_INVALID_ARG;
+    if (n >= (1ll << 40)) return SKIPARSE_ERR_UNSUPPORTED;
+    const int e = skiparse::launch_exp2(x, y, n, method, stream);
+    return e == 0 ? SKIPARSE_OK : cuda_fail(e);
+}
+
 int skiparse_get_device_status(skiparse_stream_t stream) {
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
         cudaGetLastError();
-        return SKIPARSE_ERR_CUDA;
+        return cuda_fail(e);
     }
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_skiparse_status, sizeof(int)) != cudaSuccess) {
+    e = cudaMemcpyFromSymbol(&v, g_skiparse_status, sizeof(int));
+    if (e != cudaSuccess) {
         cudaGetLastError();
-        return SKIPARSE_ERR_CUDA;
+        return cuda_fail(e);
     }
     if (v != 0) {
         const int zero = 0;
-        if (cudaMemcpyToSymbol(g_skiparse_status, &zero, sizeof(int)) != cudaSuccess) {
+        e = cudaMemcpyToSymbol(g_skiparse_status, &zero, sizeof(int));
+        if (e != cudaSuccess) {
             cudaGetLastError();
-            return SKIPARSE_ERR_CUDA;
+            return cuda_fail(e);
         }
     }
     return v;
@@ -169,7 +191,7 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.exchange(0);
     const int e = skiparse::launch_attn_fwd(p, g, stream);
-    return e == 0 ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
+    return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
 static int rearrange_common(const void* src, void* dst, int B, int T, int H, int W, int heads,
@@ -194,7 +216,7 @@ static int rearrange_common(const void* src, void* dst, int B, int T, int H, int
     p.row_chunks = static_cast<int>(row_bytes / 16);
     p.nrows = forward ? nslot : ntok;
     const int e = skiparse::launch_rearrange(p, forward, stream);
-    return e == 0 ? SKIPARSE_OK : SKIPARSE_ERR_CUDA;
+    return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
 int skiparse_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d, int P,

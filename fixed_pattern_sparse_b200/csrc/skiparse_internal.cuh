@@ -75,5 +75,6 @@ enum : int { kOk = 0, kErrTimeout = 5 };
 int launch_attn_fwd(const AttnParams& p, const Geometry& g, void* stream);
 int launch_rearrange(const RearrangeParams& p, bool forward, void* stream);
 int attn_smem_bytes(int d);
+int launch_exp2(const float* x, float* y, long long n, int method, void* stream);
 
 }  // namespace skiparse

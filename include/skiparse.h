@@ -113,6 +113,10 @@ SKIPARSE_API int skiparse_get_device_status(skiparse_stream_t stream);
 /* Static, human-readable name of a status code. Never NULL. */
 SKIPARSE_API const char* skiparse_status_string(int status);
 
+/* Message of the last CUDA failure reported as SKIPARSE_ERR_CUDA on this host thread
+ * ("no error" if none). Static storage; never NULL. */
+SKIPARSE_API const char* skiparse_last_error_string(void);
+
 /* Library version string, static. */
 SKIPARSE_API const char* skiparse_version(void);
 
@@ -131,6 +135,16 @@ SKIPARSE_API unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns
  * Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
  */
 SKIPARSE_API int skiparse_debug_inject_fault(int kind);
+
+/*
+ * Diagnostic (no counterpart on the pages): y[i] = 2^x[i] for n fp32 device values, evaluated
+ * exactly as the attention softmax does -- method 0 with the MUFU ex2.approx instruction,
+ * method 1 with the FMA-pipe degree-3 polynomial that takes part of the exponentials off the
+ * MUFU unit (inputs below -125 give about 2^-125). x and y are device pointers, n >= 0;
+ * asynchronous on `stream`. Returns SKIPARSE_OK, SKIPARSE_ERR_INVALID_ARG or SKIPARSE_ERR_CUDA.
+ */
+SKIPARSE_API int skiparse_debug_exp2(const float* x, float* y, long long n, int method,
+                                     skiparse_stream_t stream);
 
 #ifdef __cplusplus
 }
