@@ -185,6 +185,12 @@ def barrier(world: int):
         torch.distributed.barrier()
 
 
+def aggregate_tflops(flops_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of its own workload, timed as the
+    maximum over ranks."""
+    return flops_per_step * steps * world / (max_total_ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------------ CPU oracle
 
 def oracle_sample_rows(w, mode, nrows: int, group: int = 0) -> np.ndarray:
@@ -278,7 +284,7 @@ def run_ours(args):
     total_ms = starts[0].elapsed_time(ends[-1])
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
-    value = fl * args.steps * world / (total_ms / 1e3) / 1e12
+    value = aggregate_tflops(fl, args.steps, world, total_ms)
     by_mode = {MODE_NAME[m]: statistics.mean(per_launch[i] for i in range(args.steps) if i % len(modes) == j)
                for j, m in enumerate(modes) if j < args.steps}
 
@@ -310,7 +316,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        e2e = {"value": round(fl * args.e2e_steps * world / (e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        e2e = {"value": round(aggregate_tflops(fl, args.e2e_steps, world, e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2,
                "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps}
         del staging, qh, kh, vh, oh
@@ -342,8 +348,10 @@ def run_ours(args):
         bytes_fwd = (qd.numel() + y.numel()) * 2  # read real rows, write all slots
         bytes_inv = 2 * qd.numel() * 2            # read real slots, write all rows
         res = {}
+        y2 = torch.empty_like(y)
         for name, fn, nbytes in (("rearrange", lambda m: fps.skiparse_rearrange(qd, w.P, m, out=y), bytes_fwd),
-                                 ("unrearrange", lambda m: fps.skiparse_unrearrange(y, q.shape, w.P, m, out=back), bytes_inv)):
+                                 ("unrearrange", lambda m: fps.skiparse_unrearrange(y, q.shape, w.P, m, out=back), bytes_inv),
+                                 ("switch_mode", lambda m: fps.skiparse_switch_mode(y, q.shape, w.P, m, out=y2), bytes_fwd)):
             for i in range(3):
                 fn(modes[i % len(modes)])
             r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -359,7 +367,7 @@ def run_ours(args):
         res["hbm_peak_gbs"] = float(peaks["hbm_gbs"])
         res["note"] = "algorithmic bytes (read + write) per call / CUDA-event time; inputs > L2"
         rearr = res
-        del y, back
+        del y, y2, back
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the rearrange timing")
 

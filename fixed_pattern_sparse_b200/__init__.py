@@ -16,7 +16,7 @@ TOKEN_WISE = 0
 GROUP_WISE = 1
 
 __all__ = ["TOKEN_WISE", "GROUP_WISE", "SkiparseError", "skiparse2d_attn_fwd", "skiparse_rearrange",
-           "skiparse_unrearrange", "rearranged_shape", "padded_extent", "subseq_len", "class_len",
+           "skiparse_unrearrange", "skiparse_switch_mode", "rearranged_shape", "padded_extent", "subseq_len", "class_len",
            "get_device_status", "attn_fwd_from_host", "HostStaging", "attn_flops", "STATUS"]
 
 
@@ -109,6 +109,25 @@ def skiparse_unrearrange(y: torch.Tensor, shape, P: int, mode: int, out: torch.T
     B, T, H, W, heads, d = shape
     check(lib().skiparse_unrearrange(y.data_ptr(), out.data_ptr(), B, T, H, W, heads, d, P, mode,
                                      _stream_ptr(stream)), "skiparse_unrearrange")
+    return out
+
+
+def skiparse_switch_mode(y: torch.Tensor, shape, P: int, src_mode: int, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """src_mode's rearranged layout -> the other mode's rearranged layout (pads zero)."""
+    _need_cuda_bf16("y", y)
+    shape = tuple(int(s) for s in shape)
+    rshape = tuple(rearranged_shape(shape, P))
+    if tuple(y.shape) != rshape:
+        raise ValueError("y does not match the rearranged shape of `shape`")
+    if out is None:
+        out = torch.empty(rshape, dtype=torch.bfloat16, device=y.device)
+    _need_cuda_bf16("out", out)
+    if tuple(out.shape) != rshape:
+        raise ValueError(f"out must have shape {rshape}")
+    B, T, H, W, heads, d = shape
+    check(lib().skiparse_switch_mode(y.data_ptr(), out.data_ptr(), B, T, H, W, heads, d, P, src_mode,
+                                     _stream_ptr(stream)), "skiparse_switch_mode")
     return out
 
 

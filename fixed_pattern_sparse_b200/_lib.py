@@ -18,6 +18,7 @@ SIGNATURES = {
     "skiparse2d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_rearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_unrearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse_switch_mode": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_rearranged_numel": (_LL, [_I] * 7),
     "skiparse_padded_extent": (_I, [_I, _I]),
     "skiparse_subseq_len": (_LL, [_I] * 4),

@@ -1,11 +1,15 @@
-// rearrange.cu -- standalone Skiparse rearrange and inverse rearrange for B200 (sm_100a).
+// rearrange.cu -- standalone Skiparse rearrange, inverse rearrange and pattern switch for B200
+// (sm_100a).
 //
 // Summary page of OSP-Next, 方法步骤详情 (method step details): the (B,T,H,W,C) tokens are
 // rearranged into P^2 subsequences of length N/P^2 (padding H and W up to multiples of P^2),
-// and the attention result is rearranged back to the original layout. Both directions are a
-// permutation of whole token rows of heads*d bf16 values (contiguous in both layouts), so
-// the kernels are pure HBM copies: one warp moves one row with 16-byte loads and stores,
-// several chunks in flight per lane; pad rows of the rearranged tensor are written as zero.
+// and the attention result is rearranged back to the original layout; 核心方法 (core method):
+// token-wise and group-wise layers alternate, and under sequence parallelism a pattern switch is
+// a local rearrange plus one exchange -- the switch kernel here is that local step, from one
+// mode's rearranged layout straight to the other's. All three are permutations of whole token
+// rows of heads*d bf16 values (contiguous in every layout), so the kernels are pure HBM copies:
+// one warp moves one row with 16-byte loads and stores, several chunks in flight per lane; pad
+// rows of a rearranged result are written as zero.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -32,9 +36,11 @@ __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) {
                  : "memory");
 }
 
-// forward = true : row is a slot (seq*n + pos) of the rearranged tensor.
-// forward = false: row is a token ((b*T + t)*H + h)*W + w of the original tensor.
-template <bool kForward>
+// kKind 0 (rearrange): row is a slot (seq*n + pos) of the rearranged tensor (mode p.mode).
+// kKind 1 (inverse)  : row is a token ((b*T + t)*H + h)*W + w of the original tensor.
+// kKind 2 (switch)   : row is a slot of the other mode's rearranged tensor; the source is the
+//                      same token's slot in mode p.mode's rearranged tensor.
+template <int kKind>
 __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const RearrangeParams p) {
     const int lane = threadIdx.x & 31;
     const long long warp0 = (static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
@@ -45,7 +51,8 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
     for (long long row = warp0; row < p.nrows; row += nwarps) {
         long long src_row;
         bool real = true;
-        if (kForward) {
+        if (kKind == 0 || kKind == 2) {
+            const int out_mode = kKind == 0 ? p.mode : 1 - p.mode;
             const long long seq = row / p.n;
             const long long pos = row - seq * p.n;
             const int b = static_cast<int>(seq / q2);
@@ -54,10 +61,20 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
             const long long tr = pos / p.S;
             const int r = static_cast<int>(tr % p.R);
             const int t = static_cast<int>(tr / p.R);
-            const int h = axis_coord(r, c / p.P, p.P, p.mode);
-            const int w = axis_coord(s, c % p.P, p.P, p.mode);
+            const int h = axis_coord(r, c / p.P, p.P, out_mode);
+            const int w = axis_coord(s, c % p.P, p.P, out_mode);
             real = h < p.H && w < p.W;
-            src_row = ((static_cast<long long>(b) * p.T + t) * p.H + h) * p.W + w;
+            if (kKind == 0) {
+                src_row = ((static_cast<long long>(b) * p.T + t) * p.H + h) * p.W + w;
+            } else {
+                int ci = 0, r2 = 0, cj = 0, s2 = 0;
+                if (real) {
+                    axis_class(h, p.P, p.mode, ci, r2);
+                    axis_class(w, p.P, p.mode, cj, s2);
+                }
+                const long long sseq = static_cast<long long>(b) * q2 + ci * p.P + cj;
+                src_row = sseq * p.n + (static_cast<long long>(t) * p.R + r2) * p.S + s2;
+            }
         } else {
             long long tok = row;
             const int w = static_cast<int>(tok % p.W);
@@ -93,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
 
 }  // namespace
 
-int launch_rearrange(const RearrangeParams& p, bool forward, void* stream) {
+int launch_rearrange(const RearrangeParams& p, int kind, void* stream) {
     if (p.nrows <= 0) return static_cast<int>(cudaSuccess);
     int dev = 0, sms = 148;
     cudaError_t e = cudaGetDevice(&dev);
@@ -104,10 +121,12 @@ int launch_rearrange(const RearrangeParams& p, bool forward, void* stream) {
     const long long max_blocks = static_cast<long long>(sms) * 8;  // 8 x 256 threads per SM
     const int blocks = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (forward)
-        skiparse_rearrange_kernel<true><<<blocks, kThreads, 0, st>>>(p);
+    if (kind == 0)
+        skiparse_rearrange_kernel<0><<<blocks, kThreads, 0, st>>>(p);
+    else if (kind == 1)
+        skiparse_rearrange_kernel<1><<<blocks, kThreads, 0, st>>>(p);
     else
-        skiparse_rearrange_kernel<false><<<blocks, kThreads, 0, st>>>(p);
+        skiparse_rearrange_kernel<2><<<blocks, kThreads, 0, st>>>(p);
     return static_cast<int>(cudaGetLastError());
 }
 

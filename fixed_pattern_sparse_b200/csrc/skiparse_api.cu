@@ -195,7 +195,7 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
 }
 
 static int rearrange_common(const void* src, void* dst, int B, int T, int H, int W, int heads,
-                            int d, int P, int mode, skiparse_stream_t stream, bool forward) {
+                            int d, int P, int mode, skiparse_stream_t stream, int kind) {
     if (!src || !dst) return SKIPARSE_ERR_INVALID_ARG;
     Geometry g;
     int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
@@ -206,27 +206,33 @@ static int rearrange_common(const void* src, void* dst, int B, int T, int H, int
     const long long nslot = static_cast<long long>(B) * P * P * g.n;
     const size_t orig_bytes = static_cast<size_t>(ntok * row_bytes);
     const size_t rear_bytes = static_cast<size_t>(nslot * row_bytes);
-    if (forward ? overlaps(src, orig_bytes, dst, rear_bytes) : overlaps(src, rear_bytes, dst, orig_bytes))
-        return SKIPARSE_ERR_INVALID_ARG;
+    const size_t src_bytes = kind == 0 ? orig_bytes : rear_bytes;
+    const size_t dst_bytes = kind == 1 ? orig_bytes : rear_bytes;
+    if (overlaps(src, src_bytes, dst, dst_bytes)) return SKIPARSE_ERR_INVALID_ARG;
     skiparse::RearrangeParams p{};
     p.src = src;
     p.dst = dst;
     p.B = B; p.T = T; p.H = H; p.W = W; p.P = P; p.mode = mode; p.R = g.R; p.S = g.S;
     p.n = g.n;
     p.row_chunks = static_cast<int>(row_bytes / 16);
-    p.nrows = forward ? nslot : ntok;
-    const int e = skiparse::launch_rearrange(p, forward, stream);
+    p.nrows = kind == 1 ? ntok : nslot;
+    const int e = skiparse::launch_rearrange(p, kind, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
 int skiparse_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d, int P,
                        int mode, skiparse_stream_t stream) {
-    return rearrange_common(x, y, B, T, H, W, heads, d, P, mode, stream, true);
+    return rearrange_common(x, y, B, T, H, W, heads, d, P, mode, stream, 0);
 }
 
 int skiparse_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
                          int P, int mode, skiparse_stream_t stream) {
-    return rearrange_common(y, x, B, T, H, W, heads, d, P, mode, stream, false);
+    return rearrange_common(y, x, B, T, H, W, heads, d, P, mode, stream, 1);
+}
+
+int skiparse_switch_mode(const void* y_src, void* y_dst, int B, int T, int H, int W, int heads,
+                         int d, int P, int src_mode, skiparse_stream_t stream) {
+    return rearrange_common(y_src, y_dst, B, T, H, W, heads, d, P, src_mode, stream, 2);
 }
 
 }  // extern "C"

@@ -65,7 +65,7 @@ struct RearrangeParams {
     int B, T, H, W, P, mode, R, S;
     long long n;          // padded subsequence length
     int row_chunks;       // 16-byte chunks per token row (heads*d*2/16)
-    long long nrows;      // rows to write: B*P*P*n (rearrange) or B*T*H*W (unrearrange)
+    long long nrows;      // rows to write: B*P*P*n (rearrange, switch) or B*T*H*W (unrearrange)
 };
 
 // Status codes (mirror include/skiparse.h).
@@ -73,7 +73,7 @@ enum : int { kOk = 0, kErrTimeout = 5 };
 
 // Launchers (defined in the kernel translation units). They return the cudaError_t as int.
 int launch_attn_fwd(const AttnParams& p, const Geometry& g, void* stream);
-int launch_rearrange(const RearrangeParams& p, bool forward, void* stream);
+int launch_rearrange(const RearrangeParams& p, int kind, void* stream);  // 0 fwd, 1 inverse, 2 switch
 int attn_smem_bytes(int d);
 int launch_exp2(const float* x, float* y, long long n, int method, void* stream);
 

@@ -91,6 +91,20 @@ SKIPARSE_API int skiparse_rearrange(const void* x, void* y, int B, int T, int H,
 SKIPARSE_API int skiparse_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
                          int P, int mode, skiparse_stream_t stream);
 
+/*
+ * Pattern switch (核心方法: token-wise and group-wise layers alternate; under sequence
+ * parallelism a switch is a local rearrange plus one exchange -- this is that local step).
+ *   y_src : (B*P*P, n, heads, d) bf16 in src_mode's rearranged layout, read-only; its pad slots
+ *           are ignored.
+ *   y_dst : (B*P*P, n, heads, d) bf16, written entirely in the other mode's rearranged layout;
+ *           pad slots are +0.0. Must not overlap y_src.
+ * Equal, bit for bit, to skiparse_unrearrange(src_mode) followed by skiparse_rearrange of the
+ * other mode, in one pass over HBM.
+ */
+SKIPARSE_API int skiparse_switch_mode(const void* y_src, void* y_dst, int B, int T, int H, int W,
+                                      int heads, int d, int P, int src_mode,
+                                      skiparse_stream_t stream);
+
 /* Number of elements of the rearranged tensor, B*P*P*n*heads*d; -1 on invalid arguments. */
 SKIPARSE_API long long skiparse_rearranged_numel(int B, int T, int H, int W, int heads, int d, int P);
 

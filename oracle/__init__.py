@@ -12,6 +12,8 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   padded_extent, axis_map, rearrange, unrearrange -- pinned (pixel_unshuffle library
       routine, hand-derived golden class maps, permutation/identity/local-equivalence
       invariants, two-hop property);
+  switch_mode -- pinned (equals unrearrange of one mode followed by rearrange of the other;
+      a switch there and back is the identity on real slots; pads are zero);
   attn_fwd, attn_fwd_rows, masked_attention -- pinned (P=1 against fp64
       scaled_dot_product_attention, numpy brute force with an explicit 2-D mask,
       closed forms, pad invariance).
@@ -49,6 +51,8 @@ def lib():
         L.oracle_rearrange.restype = c_int
         L.oracle_unrearrange.argtypes = [vp, vp] + shape8
         L.oracle_unrearrange.restype = c_int
+        L.oracle_switch_mode.argtypes = [vp, vp] + shape8
+        L.oracle_switch_mode.restype = c_int
         L.oracle_unrearrange_f64.argtypes = [vp, vp] + shape8
         L.oracle_unrearrange_f64.restype = c_int
         L.oracle_masked_attention.argtypes = [vp, vp, vp, vp, vp, c_ll, c_ll, c_int, c_int, c_int]
@@ -121,6 +125,16 @@ def unrearrange(y, shape, P: int, mode: int):
     _check(lib().oracle_unrearrange(_ptr(yb), _ptr(x), B, T, H, W, heads, d, P, mode),
            "unrearrange")
     return x
+
+
+def switch_mode(y, shape, P: int, src_mode: int):
+    """src_mode's rearranged layout -> the other mode's rearranged layout (bit patterns)."""
+    yb = _bits(y)
+    B, T, H, W, heads, d = shape
+    out = np.empty_like(yb)
+    _check(lib().oracle_switch_mode(_ptr(yb), _ptr(out), B, T, H, W, heads, d, P, src_mode),
+           "switch_mode")
+    return out
 
 
 def unrearrange_f64(y: np.ndarray, shape, P: int, mode: int):

@@ -152,6 +152,40 @@ int oracle_unrearrange_f64(const double* y, double* x,
     return 0;
 }
 
+/* Pattern switch between layers (核心方法: token-wise and group-wise alternate between layers;
+ * 方法步骤详情: under SSP a switch is a local rearrange plus one exchange). The local step: a
+ * tensor in src_mode's rearranged layout goes straight to the other mode's rearranged layout;
+ * every real token row moves from its src_mode slot to its dst_mode slot, pad slots of the
+ * result are 0. */
+int oracle_switch_mode(const uint16_t* ysrc, uint16_t* ydst,
+                       int B, int T, int H, int W, int heads, int d, int P, int src_mode) {
+    if (check_shape(B, T, H, W, heads, d, P, src_mode)) return -1;
+    const int dst_mode = 1 - src_mode;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    const long long n = (long long)T * R * S;
+    const long long row = (long long)heads * d;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hp; ++h)
+                for (int w = 0; w < Wp; ++w) {
+                    int ci, r, cj, s;
+                    oracle_axis_map(h, P, dst_mode, &ci, &r);
+                    oracle_axis_map(w, P, dst_mode, &cj, &s);
+                    const long long dslot = ((long long)b * P * P + ci * P + cj) * n + ((long long)t * R + r) * S + s;
+                    uint16_t* dst = ydst + dslot * row;
+                    if (h < H && w < W) {
+                        oracle_axis_map(h, P, src_mode, &ci, &r);
+                        oracle_axis_map(w, P, src_mode, &cj, &s);
+                        const long long sslot = ((long long)b * P * P + ci * P + cj) * n + ((long long)t * R + r) * S + s;
+                        for (long long e = 0; e < row; ++e) dst[e] = ysrc[sslot * row + e];
+                    } else {
+                        for (long long e = 0; e < row; ++e) dst[e] = 0;
+                    }
+                }
+    return 0;
+}
+
 /* Step 2: dense softmax attention of one query row over the real keys of its own
  * subsequence (核心方法: each subsequence attends densely, which is why FlashAttention
  * runs natively; 方法步骤详情: padded keys are removed by the attention mask).

@@ -45,6 +45,11 @@ int oracle_unrearrange(const uint16_t* y, uint16_t* x,
 int oracle_unrearrange_f64(const double* y, double* x,
                            int B, int T, int H, int W, int heads, int d, int P, int mode);
 
+/* Pattern switch: ysrc in src_mode's rearranged layout -> ydst in the other mode's rearranged
+ * layout (both (B*P*P, n, heads, d)); pad slots of ydst are 0. */
+int oracle_switch_mode(const uint16_t* ysrc, uint16_t* ydst,
+                       int B, int T, int H, int W, int heads, int d, int P, int src_mode);
+
 /* Dense softmax attention inside every subsequence, with the pad-key mask, in fp64.
  * yq/yk/yv (nseq, n, heads, d) bf16 bits, valid (nseq*n), yo (nseq, n, heads, d) fp64.
  * Pad-query rows of yo are left untouched. */

@@ -118,3 +118,29 @@ def test_unrearrange_ignores_pad_slots(fps, w, mode):
     want = oracle.unrearrange(y, w.shape, w.P, mode)
     got = fps.skiparse_unrearrange(y.cuda(), w.shape, w.P, mode)
     assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("name", ["tiny", "anyres", "480p", "720p", "768p", "768p_p3"])
+@pytest.mark.parametrize("src", [TOK, GRP])
+def test_switch_mode_bit_exact(fps, name, src):
+    """Token-wise <-> group-wise re-layout in one pass, against the oracle."""
+    w = synth.WORKLOADS[name]
+    x, _, _ = synth.qkv(w)
+    ysrc = oracle.rearrange(x, w.P, src)
+    want = oracle.switch_mode(ysrc, w.shape, w.P, src)
+    yd = torch.from_numpy(ysrc.view(np.int16)).cuda().view(torch.bfloat16)
+    out = torch.empty_like(yd)
+    out.view(torch.int16).fill_(-1)  # canary: pad slots must become +0.0
+    fps.skiparse_switch_mode(yd, w.shape, w.P, src, out=out)
+    assert fps.get_device_status() == 0
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+def test_switch_mode_equals_inverse_then_rearrange(fps):
+    w = synth.custom(2, 3, 11, 17, 3, 64, 3, "p3_b2")
+    x = synth.qkv(w)[0].cuda()
+    for src in (TOK, GRP):
+        y = fps.skiparse_rearrange(x, w.P, src)
+        a = fps.skiparse_switch_mode(y, w.shape, w.P, src)
+        b = fps.skiparse_rearrange(fps.skiparse_unrearrange(y, w.shape, w.P, src), w.P, 1 - src)
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))

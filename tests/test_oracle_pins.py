@@ -357,3 +357,32 @@ def test_bad_arguments_are_rejected():
     assert L.oracle_padded_extent(0, 2) < 0 and L.oracle_padded_extent(4, 0) < 0
     with pytest.raises(RuntimeError):
         oracle.axis_map(3, 2, 7)
+
+
+# --------------------------------------------------------------- pattern-switch pins
+
+@pytest.mark.parametrize("B,T,H,W,heads,d,P", SHAPES)
+@pytest.mark.parametrize("src", [TOK, GRP])
+def test_switch_mode_is_unrearrange_then_rearrange(B, T, H, W, heads, d, P, src):
+    """核心方法: the two modes alternate between layers; the switch of one tensor between the
+    modes' layouts is the inverse rearrange of one followed by the rearrange of the other."""
+    x = random_bits((B, T, H, W, heads, d), 500 + P + src)
+    ysrc = oracle.rearrange(x, P, src)
+    got = oracle.switch_mode(ysrc, x.shape, P, src)
+    want = oracle.rearrange(oracle.unrearrange(ysrc, x.shape, P, src), P, 1 - src)
+    assert np.array_equal(got, want)
+    # and back again gives the source layout (its pad slots are zero already)
+    assert np.array_equal(oracle.switch_mode(got, x.shape, P, 1 - src), ysrc)
+
+
+def test_switch_mode_ignores_source_pad_slots():
+    w = synth.WORKLOADS["anyres"]
+    x, _, _ = synth.qkv(w)
+    y, valid = oracle.rearrange(x, w.P, TOK, with_valid=True)
+    junk = y.copy()
+    junk[valid == 0] = 0x4000
+    a = oracle.switch_mode(y, w.shape, w.P, TOK)
+    b = oracle.switch_mode(junk, w.shape, w.P, TOK)
+    assert np.array_equal(a, b)
+    _, gvalid = oracle.rearrange(x, w.P, GRP, with_valid=True)
+    assert np.all(a[gvalid == 0] == 0)
