@@ -53,7 +53,8 @@ KNOWN_TRAFFIC = {
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
                 "fixed_pattern_sparse_b200/csrc/ptx_sm100.cuh",
-                "fixed_pattern_sparse_b200/csrc/skiparse_internal.cuh"]
+                "fixed_pattern_sparse_b200/csrc/skiparse_internal.cuh",
+                "fixed_pattern_sparse_b200/csrc/attn_common.cuh"]
 
 
 def kernel_hash() -> str:
@@ -409,6 +410,76 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+# ------------------------------------------------------------- hybrid stack harness
+
+def stack_schedule(layers: int, dense_front: int, dense_back: int):
+    """(P, mode) per layer of a hybrid stack: dense (P=1) blocks at both ends, Skiparse-2D in
+    the middle with token-wise and group-wise layers alternating (summary page 核心方法 /
+    实验结果: 4 full-attention blocks at the front and 4 at the back, the rest sparse)."""
+    sched, k = [], 0
+    for i in range(layers):
+        if i < dense_front or i >= layers - dense_back:
+            sched.append((1, 0))
+        else:
+            sched.append((None, k % 2))
+            k += 1
+    return sched
+
+
+def run_stack(args):
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_pg(world, "nccl")
+    import fixed_pattern_sparse_b200 as fps
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = (t.to(dev) for t in synth.qkv(w))
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    hybrid = [(w.P if p is None else p, m) for p, m in stack_schedule(args.layers, args.dense_front, args.dense_back)]
+    dense = [(1, 0)] * args.layers
+
+    def one_pass(sched):
+        for P, mode in sched:
+            fps.skiparse2d_attn_fwd(q, k, v, P, mode, out=out)
+
+    def timed(sched, steps):
+        one_pass(sched)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one_pass(sched)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+
+    for _ in range(args.warmup):
+        one_pass(hybrid)
+    h_ms = timed(hybrid, args.steps)
+    d_ms = timed(dense, max(1, args.steps // 2))
+    if fps.get_device_status() != 0:
+        raise SystemExit("device status error in the stack timing")
+    fl_h = sum(flops_padded(synth.custom(w.B, w.T, w.H, w.W, w.heads, w.d, P)) for P, _ in hybrid)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "hybrid attention stack: ms per pass vs an all-dense stack (attention layers only)",
+            "value": round(h_ms, 2), "unit": "ms", "higher_is_better": False, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "scaling": "weak", "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, the same inputs for every layer",
+            "config": {"workload": describe(w), "layers": args.layers,
+                       "dense_front": args.dense_front, "dense_back": args.dense_back,
+                       "sparse_layers": args.layers - args.dense_front - args.dense_back,
+                       "sparse_modes": "alternating token-wise / group-wise"},
+            "dense_stack_ms": round(d_ms, 2), "attention_speedup": round(d_ms / h_ms, 3),
+            "hybrid_tflops": round(fl_h / (h_ms / 1e3) / 1e12, 1), "gpu_launches_per_pass": args.layers,
+        }), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 # --------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -475,11 +546,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rearrange", action="store_true")
     ap.add_argument("--rearrange-steps", type=int, default=10)
+    ap.add_argument("--stack", action="store_true",
+                    help="time a hybrid stack of dense and alternating Skiparse-2D layers instead")
+    ap.add_argument("--layers", type=int, default=40)
+    ap.add_argument("--dense-front", type=int, default=4)
+    ap.add_argument("--dense-back", type=int, default=4)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.stack:
+        run_stack(args)
     else:
         run_ours(args)
 

@@ -17,7 +17,8 @@ GROUP_WISE = 1
 
 __all__ = ["TOKEN_WISE", "GROUP_WISE", "SkiparseError", "skiparse2d_attn_fwd", "skiparse_rearrange",
            "skiparse_unrearrange", "skiparse_switch_mode", "rearranged_shape", "padded_extent", "subseq_len", "class_len",
-           "get_device_status", "attn_fwd_from_host", "HostStaging", "attn_flops", "STATUS"]
+           "get_device_status", "attn_fwd_from_host", "HostStaging", "attn_flops", "STATUS",
+           "skiparse2d_attn_fwd_lse", "skiparse2d_attn_bwd", "SkiparseAttention", "skiparse_attention"]
 
 
 def _stream_ptr(stream) -> int:
@@ -76,6 +77,73 @@ def skiparse2d_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: in
                                     B, T, H, W, heads, d, P, mode, _stream_ptr(stream)),
           "skiparse2d_attn_fwd")
     return out
+
+
+def skiparse2d_attn_fwd_lse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, P: int, mode: int,
+                            out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Forward that also returns lse (B,T,H,W,heads) fp32, the natural-log log-sum-exp of
+    q.k/sqrt(d) over each token's class, for the backward pass."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda_bf16(name, t)
+    if q.dim() != 6 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one (B,T,H,W,heads,d) shape")
+    out = torch.empty_like(q) if out is None else out
+    _need_cuda_bf16("out", out)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    if lse is None:
+        lse = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(q.shape[:5]) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 (B,T,H,W,heads) tensor")
+    B, T, H, W, heads, d = q.shape
+    check(lib().skiparse2d_attn_fwd_lse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                        B, T, H, W, heads, d, P, mode, _stream_ptr(stream)),
+          "skiparse2d_attn_fwd_lse")
+    return out, lse
+
+
+def skiparse2d_attn_bwd(q, k, v, out, dout, lse, P: int, mode: int, dq=None, dk=None, dv=None, delta=None,
+                        stream=None):
+    """Backward pass: returns (dq, dk, dv), bf16 (B,T,H,W,heads,d). `delta` is an optional fp32
+    (B,T,H,W,heads) workspace (allocated here when not given)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _need_cuda_bf16(name, t)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} must have q's shape")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(q.shape[:5]) or not lse.is_cuda:
+        raise ValueError("lse must be a CUDA fp32 (B,T,H,W,heads) tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    delta = torch.empty(q.shape[:5], dtype=torch.float32, device=q.device) if delta is None else delta
+    B, T, H, W, heads, d = q.shape
+    check(lib().skiparse2d_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta.data_ptr(),
+                                    B, T, H, W, heads, d, P, mode, _stream_ptr(stream)), "skiparse2d_attn_bwd")
+    return dq, dk, dv
+
+
+class SkiparseAttention(torch.autograd.Function):
+    """Differentiable Skiparse-2D attention: forward and backward both run the sm_100a kernels."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, P: int, mode: int):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        out, lse = skiparse2d_attn_fwd_lse(q, k, v, P, mode)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.P, ctx.mode = P, mode
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = skiparse2d_attn_bwd(q, k, v, out, dout.contiguous(), lse, ctx.P, ctx.mode)
+        return dq, dk, dv, None, None
+
+
+def skiparse_attention(q, k, v, P: int, mode: int):
+    """Autograd-aware Skiparse-2D attention on (B,T,H,W,heads,d) bf16 CUDA tensors."""
+    return SkiparseAttention.apply(q, k, v, P, mode)
 
 
 def skiparse_rearrange(x: torch.Tensor, P: int, mode: int, out: torch.Tensor | None = None,

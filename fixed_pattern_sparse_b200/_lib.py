@@ -16,6 +16,8 @@ LIB_PATH = os.path.join(HERE, "libskiparse.so")
 _I, _LL, _ULL, _VP, _CP = ctypes.c_int, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_char_p
 SIGNATURES = {
     "skiparse2d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse2d_attn_fwd_lse": (_I, [_VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse2d_attn_bwd": (_I, [_VP] * 10 + [_I] * 8 + [_VP]),
     "skiparse_rearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_unrearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_switch_mode": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),

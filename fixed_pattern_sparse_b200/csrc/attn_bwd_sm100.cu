@@ -1,0 +1,454 @@
+// attn_bwd_sm100.cu -- backward pass of the fused Skiparse-2D attention for B200 (sm_100a).
+//
+// For one (b, class, head) subsequence of real tokens (summary page of OSP-Next, 核心方法 /
+// 方法步骤详情: dense softmax attention inside each class), with P = softmax(Q K^T / sqrt(d))
+// recomputed from the forward's log-sum-exp L and D_i = dO_i . O_i:
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - D),   dQ = dS K / sqrt(d),   dK = dS^T Q / sqrt(d).
+// Three launches, all reading and writing the original (B,T,H,W,heads,d) layout through the
+// class geometry (nothing rearranged is materialised):
+//   1. delta kernel: D = rowsum(dO o O) for every (token, head) row (HBM-bound);
+//   2. key-major kernel (KV = true): a CTA keeps one 128-key tile (K, V) and streams the class's
+//      query tiles (Q, dO, L, D): S^T = K Q^T and dP^T = V dO^T into TMEM; softmax warps make
+//      P^T and dS^T (bf16, over their own TMEM columns); dV += P^T dO and dK += dS^T Q accumulate
+//      in TMEM (TMEM: S^T, dP^T, dV, dK = 512 columns);
+//   3. query-major kernel (KV = false): a CTA keeps one 128-query tile (Q, dO, L, D) and streams
+//      the class's key tiles (K, V): S, dP into TMEM, dS, then dQ += dS K in TMEM.
+// No atomics: every gradient row is produced by exactly one CTA, so results are deterministic.
+// Warp roles (11 warps): two softmax warpgroups (each owns 64 of the 128 streamed columns of
+// every TMEM row), two producer warps (16-byte cp.async gathers of class rows into the UMMA
+// swizzled layout, 4-byte cp.async for L and D), one MMA warp (tcgen05.mma, one thread).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "attn_common.cuh"
+
+namespace skiparse {
+namespace {
+
+constexpr int kBwdThreads = 352;
+constexpr int kBwdProd0 = 8;
+constexpr int kBwdProducers = 64;
+constexpr int kBwdMma = 10;
+constexpr int kBwdSoftmax = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, bool KV>
+struct BwdCfg : TileGeom<D> {
+    using G = TileGeom<D>;
+    using G::SW;
+    using G::BOX_BYTES;
+    using G::TILE_BYTES;
+    using G::LAYOUT;
+    using G::KSTEPS;
+    // shared memory: two stationary tiles, two streamed slots of two tiles, L/D vectors
+    static constexpr int OFF_A1 = 0;
+    static constexpr int OFF_A2 = TILE_BYTES;
+    static constexpr int OFF_B = 2 * TILE_BYTES;              // slot s: B1 at +2sT, B2 at +(2s+1)T
+    static constexpr int OFF_VEC = OFF_B + 4 * TILE_BYTES;    // [slot or stationary][L,D][128] fp32
+    static constexpr int VEC_BYTES = 2 * 2 * kTileRows * 4;
+    static constexpr int OFF_BAR = OFF_VEC + VEC_BYTES;
+    static constexpr int B_STAT = 0, B_FULL = 1, B_EMPTY = 3, B_X1 = 5, B_X2 = 6, B_P = 7, B_DS = 8,
+                         B_ACC = 9, B_DRAIN = 10, NBARS = 11;
+    static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
+    static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+    static constexpr int SMEM_USED = OFF_ABORT + 4;
+    static constexpr int SMEM_BYTES = SMEM_USED + 1024 > 118784 ? SMEM_USED + 1024 : 118784;
+    static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+    static constexpr uint32_t COL_X1 = 0, COL_X2 = 128, COL_ACC1 = 256, COL_ACC2 = 256 + D, NCOLS = 512;
+    static_assert(COL_ACC2 + D <= NCOLS, "TMEM overflow");
+};
+
+// TMEM column of K-step kk (16 streamed rows) of a bf16 operand written by the two softmax
+// warpgroups over their own halves of a 128-column score region: rows 0..63 -> columns 0..31,
+// rows 64..127 -> columns 64..95.
+__device__ __forceinline__ uint32_t half_packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+
+// 4-byte cp.async of one fp32 per tile row (L or D of the row's token and head).
+__device__ __forceinline__ void load_vec(uint32_t dst, const float* __restrict__ src, const RowMap& rows,
+                                         int first, int n_c, int pw, int lane) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int r = 64 * pw + 32 * half + lane;
+        int i = first + r;
+        i = i < n_c ? i : n_c - 1;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4u * r),
+                     "l"(src + rows(i))
+                     : "memory");
+    }
+}
+
+template <int D, bool KV>
+__global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const BwdParams p) {
+    using C = BwdCfg<D, KV>;
+    const int tile = blockIdx.x;
+    const int head = blockIdx.y;
+    const int seq = blockIdx.z;
+    const int q2 = p.P * p.P;
+    const int b = seq / q2, c = seq % q2, ci = c / p.P, cj = c % p.P;
+    const int Rc = p.Rc[ci], Sc = p.Sc[cj];
+    const int n_c = p.T * Rc * Sc;
+    const int first = tile * kTileRows;
+    if (first >= n_c) return;  // uniform over the CTA, before any shared state
+    const int nstream = (n_c + kTileRows - 1) / kTileRows;
+    const RowMap rows{p.T, p.H, p.W, p.heads, p.P, p.mode, ci, cj, Rc, Sc, b, head};
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_base & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t sbase = raw_base + pad;
+    auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+    const float* vecs = reinterpret_cast<const float*>(smem + C::OFF_VEC);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t lim = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar(C::B_STAT), kBwdProducers);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(bar(C::B_FULL + s), kBwdProducers);
+            ptx::mbar_init(bar(C::B_EMPTY + s), 1);
+        }
+        ptx::mbar_init(bar(C::B_X1), 1);
+        ptx::mbar_init(bar(C::B_X2), 1);
+        ptx::mbar_init(bar(C::B_P), kBwdSoftmax);
+        ptx::mbar_init(bar(C::B_DS), kBwdSoftmax);
+        ptx::mbar_init(bar(C::B_ACC), 1);
+        ptx::mbar_init(bar(C::B_DRAIN), 1);
+        *abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kBwdMma) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::NCOLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // stationary tiles: (K, V) for the key-major kernel, (Q, dO) for the query-major one
+    const uint16_t* g_a1 = KV ? p.k : p.q;
+    const uint16_t* g_a2 = KV ? p.v : p.dout;
+    const uint16_t* g_b1 = KV ? p.q : p.k;
+    const uint16_t* g_b2 = KV ? p.dout : p.v;
+
+    if (warp == kBwdProd0 || warp == kBwdProd0 + 1) {
+        // ------------------------------------------------------------------ producers
+        const int pw = warp - kBwdProd0;
+        load_tile<D>(sbase + C::OFF_A1, g_a1, rows, first, n_c, pw, lane);
+        load_tile<D>(sbase + C::OFF_A2, g_a2, rows, first, n_c, pw, lane);
+        if (!KV) {  // the stationary queries' L and D
+            load_vec(sbase + C::OFF_VEC, p.lse, rows, first, n_c, pw, lane);
+            load_vec(sbase + C::OFF_VEC + 4 * kTileRows, p.delta, rows, first, n_c, pw, lane);
+        }
+        cp_async_commit();
+        uint32_t prev_bar = bar(C::B_STAT);
+        bool ok = true;
+        for (int j = 0; j < nstream; ++j) {
+            const int s = j & 1;
+            if (j >= 2) {
+                int w_ok = 1;
+                if (lane == 0) w_ok = ptx::mbar_wait(bar(C::B_EMPTY + s), ((j >> 1) - 1) & 1, abort, lim);
+                w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+                if (!w_ok) {
+                    ok = false;
+                    break;
+                }
+            }
+            const uint32_t slot = sbase + C::OFF_B + 2 * s * C::TILE_BYTES;
+            load_tile<D>(slot, g_b1, rows, j * kTileRows, n_c, pw, lane);
+            load_tile<D>(slot + C::TILE_BYTES, g_b2, rows, j * kTileRows, n_c, pw, lane);
+            if (KV) {  // the streamed queries' L and D
+                const uint32_t v = sbase + C::OFF_VEC + s * 2 * 4 * kTileRows;
+                load_vec(v, p.lse, rows, j * kTileRows, n_c, pw, lane);
+                load_vec(v + 4 * kTileRows, p.delta, rows, j * kTileRows, n_c, pw, lane);
+            }
+            cp_async_commit();
+            cp_async_wait<1>();
+            fence_proxy_async();
+            ptx::mbar_arrive(prev_bar);
+            prev_bar = bar(C::B_FULL + s);
+        }
+        cp_async_wait<0>();
+        if (ok) {
+            fence_proxy_async();
+            ptx::mbar_arrive(prev_bar);
+        } else {
+            record_abort(abort, p.status);
+        }
+    } else if (warp == kBwdMma) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_x = ptx::idesc_bf16_f32(kTileRows, kTileRows, false);
+            const uint32_t idesc_acc = ptx::idesc_bf16_f32(kTileRows, D, true);
+            const uint64_t a1 = ptx::smem_desc(sbase + C::OFF_A1, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t a2 = ptx::smem_desc(sbase + C::OFF_A2, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t bk0 = ptx::smem_desc(sbase + C::OFF_B, 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t bm0 = ptx::smem_desc(sbase + C::OFF_B, C::BOX_BYTES, 8 * C::SW, C::LAYOUT);
+            auto x_mma = [&](uint64_t a, uint64_t bk, uint32_t d_tmem) {   // D = A B^T over d
+#pragma unroll
+                for (int kk = 0; kk < C::KSTEPS; ++kk) {
+                    const uint32_t off = C::kstep_off(kk) >> 4;
+                    ptx::mma_ss(d_tmem, a + off, bk + off, idesc_x, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto acc_mma = [&](uint32_t a_col, uint64_t bm, uint32_t d_tmem, bool acc) {  // D += A B
+#pragma unroll
+                for (int kk = 0; kk < kTileRows / 16; ++kk)
+                    ptx::mma_ts(d_tmem, tmem + a_col + half_packed_col(kk), bm + ((kk * 16 * C::SW) >> 4),
+                                idesc_acc, (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = ptx::mbar_wait(bar(C::B_STAT), 0, abort, lim);
+            for (int j = 0; ok && j < nstream; ++j) {
+                const int s = j & 1;
+                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint64_t b1k = bk0 + ((2 * s * C::TILE_BYTES) >> 4);
+                const uint64_t b2k = bk0 + (((2 * s + 1) * C::TILE_BYTES) >> 4);
+                const uint64_t b1m = bm0 + ((2 * s * C::TILE_BYTES) >> 4);
+                const uint64_t b2m = bm0 + (((2 * s + 1) * C::TILE_BYTES) >> 4);
+                x_mma(a1, b1k, tmem + C::COL_X1);
+                ptx::mma_commit(bar(C::B_X1));
+                x_mma(a2, b2k, tmem + C::COL_X2);
+                ptx::mma_commit(bar(C::B_X2));
+                if (KV) {
+                    if (!ptx::mbar_wait(bar(C::B_P), j & 1, abort, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    acc_mma(C::COL_X1, b2m, tmem + C::COL_ACC1, j > 0);   // dV += P^T dO
+                }
+                if (!ptx::mbar_wait(bar(C::B_DS), j & 1, abort, lim)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                // key-major: dK += dS^T Q ; query-major: dQ += dS K
+                acc_mma(C::COL_X2, b1m, tmem + (KV ? C::COL_ACC2 : C::COL_ACC1), j > 0);
+                ptx::mma_commit(bar(C::B_EMPTY + s));
+            }
+            if (ok) {
+                ptx::mma_commit(bar(C::B_ACC));
+            } else {
+                record_abort(abort, p.status);
+            }
+            ptx::mma_commit(bar(C::B_DRAIN));
+            volatile int never = 0;
+            ptx::mbar_wait(bar(C::B_DRAIN), 0, &never, lim);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ softmax halves
+        const int h = warp >> 2;                        // streamed columns [64h, 64h+64)
+        const int row = threadIdx.x & 127;              // TMEM lane == stationary row
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t x1 = tmem + lane_base + C::COL_X1 + 64 * h;
+        const uint32_t x2 = tmem + lane_base + C::COL_X2 + 64 * h;
+        const float sl2 = p.scale_log2;
+        float row_l2 = 0.f, row_d = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nstream; ++j) {
+            const int s = j & 1;
+            const int valid = n_c - j * kTileRows;     // streamed rows in this tile (>= 1)
+            if (!ptx::mbar_wait(bar(C::B_X1), j & 1, abort, lim)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            // the L/D vectors were written by the producers' cp.async: observe their barrier too
+            if (!ptx::mbar_wait(KV ? bar(C::B_FULL + s) : bar(C::B_STAT), KV ? (j >> 1) & 1 : 0, abort, lim)) {
+                ok = false;
+                break;
+            }
+            if (!KV && j == 0) {
+                row_l2 = vecs[row] * kLog2e;
+                row_d = vecs[kTileRows + row];
+            }
+            const float* col_l = vecs + s * 2 * kTileRows + 64 * h;   // key-major: per column
+            const float* col_d = col_l + kTileRows;
+            float pr[64];
+            {
+                uint32_t xv[64];
+                ptx::tmem_ld32(x1, *reinterpret_cast<uint32_t(*)[32]>(&xv[0]));
+                ptx::tmem_ld32(x1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&xv[32]));
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const float l2 = KV ? col_l[e] * kLog2e : row_l2;
+                    const float pe = ptx::ex2_approx(fmaf(__uint_as_float(xv[e]), sl2, -l2));
+                    pr[e] = (64 * h + e < valid) ? pe : 0.f;   // fake (clamped) streamed rows: 0
+                }
+            }
+            if (KV) {  // P^T for dV += P^T dO
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = ptx::pack_bf16x2(pr[32 * g + 2 * e], pr[32 * g + 2 * e + 1]);
+                    ptx::tmem_st16(x1 + 16 * g, pk);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(bar(C::B_P));
+            }
+            if (!ptx::mbar_wait(bar(C::B_X2), j & 1, abort, lim)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                uint32_t dv[32];
+                ptx::tmem_ld32(x2 + 32 * g, dv);
+                ptx::tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int e0 = 32 * g + 2 * e;
+                    const float d0 = KV ? col_d[e0] : row_d, d1 = KV ? col_d[e0 + 1] : row_d;
+                    const float s0 = pr[e0] * (__uint_as_float(dv[2 * e]) - d0);
+                    const float s1 = pr[e0 + 1] * (__uint_as_float(dv[2 * e + 1]) - d1);
+                    pk[e] = ptx::pack_bf16x2(s0, s1);
+                }
+                ptx::tmem_st16(x2 + 16 * g, pk);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar(C::B_DS));
+        }
+        if (ok && ptx::mbar_wait(bar(C::B_ACC), 0, abort, lim)) {
+            ptx::tc_fence_after();
+            const int si = first + row;                 // stationary row (key or query)
+            const size_t grow = si < n_c ? static_cast<size_t>(rows(si)) : 0;
+            constexpr int HALF = D / 2;                 // accumulator columns of this warpgroup
+            // key-major: acc1 = dV (unscaled), acc2 = dK ; query-major: acc1 = dQ
+#pragma unroll
+            for (int which = 0; which < (KV ? 2 : 1); ++which) {
+                const uint32_t acc = tmem + lane_base + (which ? C::COL_ACC2 : C::COL_ACC1) + HALF * h;
+                const float mul = (KV && which == 0) ? 1.f : p.scale;
+                uint16_t* out = KV ? (which ? p.dk : p.dv) : p.dq;
+#pragma unroll
+                for (int g = 0; g < HALF / 16; ++g) {
+                    uint32_t av[16];
+                    ptx::tmem_ld16(acc + 16 * g, av);
+                    ptx::tmem_wait_ld();
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        pk[e] = ptx::pack_bf16x2(__uint_as_float(av[2 * e]) * mul, __uint_as_float(av[2 * e + 1]) * mul);
+                    if (si < n_c) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + grow * D + HALF * h + 16 * g);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
+                }
+            }
+        } else if (!*abort) {
+            record_abort(abort, p.status);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kBwdMma) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, C::NCOLS);
+    }
+}
+
+// D[row] = sum_e dO[row][e] * O[row][e]; 16 lanes per 256-byte row (fewer for smaller d).
+template <int D>
+__global__ void __launch_bounds__(256) skiparse_bwd_delta_kernel(const uint16_t* __restrict__ o,
+                                                                 const uint16_t* __restrict__ dout,
+                                                                 float* __restrict__ delta, long long nrows) {
+    constexpr int LPR = D / 8;            // lanes per row (8 bf16 = 16 bytes per lane)
+    constexpr int RPW = 32 / LPR;         // rows per warp step
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long r0 = warp0 * RPW; r0 < nrows; r0 += nwarps * RPW) {
+        const long long r = r0 + lane / LPR;
+        float acc = 0.f;
+        if (r < nrows) {
+            const uint4 a = *reinterpret_cast<const uint4*>(o + r * D + (lane % LPR) * 8);
+            const uint4 g = *reinterpret_cast<const uint4*>(dout + r * D + (lane % LPR) * 8);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+                acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(gv[e] & 0xffff0000u), acc);
+            }
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (r < nrows && lane % LPR == 0) delta[r] = acc;
+    }
+}
+
+template <int D, bool KV>
+int launch_bwd_d(const BwdParams& p, const Geometry& g, cudaStream_t stream) {
+    using C = BwdCfg<D, KV>;
+    static int attr_done_dev[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    if (dev >= 0 && dev < 64 && !attr_done_dev[dev]) {
+        e = cudaFuncSetAttribute(skiparse_attn_bwd_kernel<D, KV>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return static_cast<int>(e);
+        attr_done_dev[dev] = 1;
+    }
+    int n_max = 0;
+    for (int ci = 0; ci < g.P; ++ci)
+        for (int cj = 0; cj < g.P; ++cj) {
+            const int n_c = g.T * g.Rc[ci] * g.Sc[cj];
+            n_max = n_c > n_max ? n_c : n_max;
+        }
+    dim3 grid((n_max + kTileRows - 1) / kTileRows, g.heads, g.B * g.P * g.P);
+    skiparse_attn_bwd_kernel<D, KV><<<grid, kBwdThreads, C::SMEM_BYTES, stream>>>(p);
+    return static_cast<int>(cudaGetLastError());
+}
+
+template <int D>
+int launch_delta_d(const BwdParams& p, long long nrows, cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long rows_per_block = 8LL * (32 / (D / 8));
+    long long blocks = (nrows + rows_per_block - 1) / rows_per_block;
+    if (blocks > 16LL * sms) blocks = 16LL * sms;
+    skiparse_bwd_delta_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.out, p.dout, p.delta, nrows);
+    return static_cast<int>(cudaGetLastError());
+}
+
+template <int D>
+int launch_bwd_all(const BwdParams& p, const Geometry& g, cudaStream_t st) {
+    const long long nrows = static_cast<long long>(g.B) * g.T * g.H * g.W * g.heads;
+    int e = launch_delta_d<D>(p, nrows, st);
+    if (e) return e;
+    e = launch_bwd_d<D, true>(p, g, st);
+    if (e) return e;
+    return launch_bwd_d<D, false>(p, g, st);
+}
+
+}  // namespace
+
+int launch_attn_bwd(const BwdParams& p, const Geometry& g, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (g.d) {
+        case 32: return launch_bwd_all<32>(p, g, st);
+        case 64: return launch_bwd_all<64>(p, g, st);
+        case 128: return launch_bwd_all<128>(p, g, st);
+        default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+}
+
+}  // namespace skiparse

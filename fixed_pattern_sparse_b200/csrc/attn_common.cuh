@@ -1,0 +1,97 @@
+// attn_common.cuh -- pieces shared by the Skiparse attention kernels (forward and backward):
+// tile geometry of the UMMA canonical K-major layout, the class-local-token -> global-row map,
+// and the producers' 16-byte cp.async gather of class rows into that layout.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx_sm100.cuh"
+#include "skiparse_internal.cuh"
+
+namespace skiparse {
+
+constexpr int kTileRows = 128;  // rows of a Q/K/V tile == TMEM lanes
+
+// A 128-row tile of d bf16 columns in shared memory: boxes of 128 rows x (swizzle span) bytes,
+// 128-byte swizzle (64-byte for d = 32), 1024-byte aligned -- the canonical K-major layout
+// that tcgen05 shared-memory descriptors describe (and, read the other way, MN-major).
+template <int D>
+struct TileGeom {
+    static constexpr int SW = D >= 64 ? 128 : 64;         // swizzle span == bytes per box row
+    static constexpr int NBOX = D * 2 / SW;               // 64-/32-column boxes per row
+    static constexpr int BOX_BYTES = kTileRows * SW;      // one 128-row box
+    static constexpr int TILE_BYTES = BOX_BYTES * NBOX;   // 128 rows x D bf16
+    static constexpr uint32_t LAYOUT = SW == 128 ? 2u : 4u;  // descriptor swizzle code
+    static constexpr int KSTEPS = D / 16;                 // MMA K-steps over d
+    static constexpr int KPB = (SW / 2) / 16;             // K-steps per box
+    static_assert(D == 32 || D == 64 || D == 128, "d must be 32, 64 or 128");
+    // byte offset of K-step kk (16 columns) inside a K-major tile
+    static constexpr uint32_t kstep_off(int kk) { return (kk / KPB) * BOX_BYTES + (kk % KPB) * 32; }
+};
+
+// Global row (token*heads + head) of the class-local real token i of (b, ci, cj).
+struct RowMap {
+    int T, H, W, heads, P, mode;
+    int ci, cj, Rc, Sc, b, head;
+    __device__ __forceinline__ int operator()(int i) const {
+        const int s = i % Sc;
+        const int tr = i / Sc;
+        const int r = tr % Rc;
+        const int t = tr / Rc;
+        const int h = axis_coord(r, ci, P, mode);
+        const int w = axis_coord(s, cj, P, mode);
+        return (((b * T + t) * H + h) * W + w) * heads + head;
+    }
+};
+
+__device__ __forceinline__ void record_abort(volatile int* abort, int* status) {
+    *abort = 1;
+    atomicExch(status, kErrTimeout);
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Issues the cp.async copies of tile rows [first, first+128) of the class's real-token list
+// (rows past n_c repeat row n_c-1; they are masked or never stored) into a 128-row tile laid
+// out as the UMMA canonical K-major layout with 128-byte (64-byte for d = 32) swizzle.
+// Producer warp pw (0/1) copies tile rows [64*pw, 64*pw+64); 16 consecutive lanes cover one
+// 256-byte row so every warp instruction reads whole rows.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restrict__ g,
+                                          const RowMap& rows, int first, int n_c, int pw, int lane) {
+    using C = TileGeom<D>;
+    constexpr int CPR = D * 2 / 16;   // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;     // rows per warp instruction
+    constexpr int NI = 64 / RPI;      // warp instructions per producer warp
+    int ia = first + 64 * pw + lane, ib = ia + 32;
+    ia = ia < n_c ? ia : n_c - 1;
+    ib = ib < n_c ? ib : n_c - 1;
+    const int ra = rows(ia), rb = rows(ib);
+    const int c = lane % CPR;
+    const int rsub = lane / CPR;
+    const uint32_t box = static_cast<uint32_t>((c * 16) / C::SW);
+    const uint32_t cb = static_cast<uint32_t>(((c * 16) % C::SW) / 16);
+#pragma unroll
+    for (int k = 0; k < NI; ++k) {
+        const int rl = k * RPI + rsub;  // 0..63
+        const int grow = __shfl_sync(0xffffffffu, (k * RPI < 32) ? ra : rb, rl & 31);
+        const int r = 64 * pw + rl;     // tile row 0..127
+        const uint32_t sw = C::SW == 128 ? (cb ^ static_cast<uint32_t>(r & 7))
+                                         : (cb ^ static_cast<uint32_t>((r >> 1) & 3));
+        const uint32_t d = dst + box * C::BOX_BYTES + static_cast<uint32_t>(r) * C::SW + sw * 16u;
+        cp_async_16(d, g + static_cast<size_t>(grow) * D + c * 8);
+    }
+}
+
+
+}  // namespace skiparse

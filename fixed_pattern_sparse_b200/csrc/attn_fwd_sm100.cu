@@ -27,8 +27,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include "ptx_sm100.cuh"
-#include "skiparse_internal.cuh"
+#include "attn_common.cuh"
 
 namespace skiparse {
 namespace {
@@ -65,15 +64,16 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by mo
 constexpr unsigned kEmuMask = SKIPARSE_EMU_MASK;
 
 template <int D>
-struct Cfg {
-    static constexpr int SW = D >= 64 ? 128 : 64;         // swizzle span == bytes per box row
-    static constexpr int NBOX = D * 2 / SW;               // 64-/32-column boxes per row
-    static constexpr int BOX_BYTES = kBM * SW;            // one 128-row box
-    static constexpr int TILE_BYTES = BOX_BYTES * NBOX;   // 128 rows x D bf16
+struct Cfg : TileGeom<D> {
+    using G = TileGeom<D>;
+    using G::SW;
+    using G::NBOX;
+    using G::BOX_BYTES;
+    using G::TILE_BYTES;
+    using G::LAYOUT;
+    using G::KSTEPS;
+    using G::KPB;
     static constexpr int KST = 2, VST = 2;                // K and V ring slots
-    static constexpr uint32_t LAYOUT = SW == 128 ? 2u : 4u;  // descriptor swizzle code
-    static constexpr int KSTEPS = D / 16;                 // MMA K-steps of Q*K^T
-    static constexpr int KPB = (SW / 2) / 16;             // K-steps per box
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
     static constexpr uint32_t NCOLS = 512;
     static constexpr int OFF_Q = 0;                       // Q0, Q1
@@ -98,72 +98,9 @@ struct Cfg {
     // + slack for 1024-byte alignment; at least 116 KB so that one CTA (and its 512 TMEM
     // columns) owns an SM even for small d
     static constexpr int SMEM_BYTES = SMEM_USED + 1024 > 118784 ? SMEM_USED + 1024 : 118784;
-    static_assert(D == 32 || D == 64 || D == 128, "d must be 32, 64 or 128");
     static_assert(COL_O1 + D <= NCOLS, "TMEM overflow");
     static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
-
-// Global row (token*heads + head) of the class-local real token i of (b, ci, cj).
-struct RowMap {
-    int T, H, W, heads, P, mode;
-    int ci, cj, Rc, Sc, b, head;
-    __device__ __forceinline__ int operator()(int i) const {
-        const int s = i % Sc;
-        const int tr = i / Sc;
-        const int r = tr % Rc;
-        const int t = tr / Rc;
-        const int h = axis_coord(r, ci, P, mode);
-        const int w = axis_coord(s, cj, P, mode);
-        return (((b * T + t) * H + h) * W + w) * heads + head;
-    }
-};
-
-__device__ __forceinline__ void record_abort(volatile int* abort, int* status) {
-    *abort = 1;
-    atomicExch(status, kErrTimeout);
-}
-
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Issues the cp.async copies of tile rows [first, first+128) of the class's real-token list
-// (rows past n_c repeat row n_c-1; they are masked or never stored) into a 128-row tile laid
-// out as the UMMA canonical K-major layout with 128-byte (64-byte for d = 32) swizzle.
-// Producer warp pw (0/1) copies tile rows [64*pw, 64*pw+64); 16 consecutive lanes cover one
-// 256-byte row so every warp instruction reads whole rows.
-template <int D>
-__device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restrict__ g,
-                                          const RowMap& rows, int first, int n_c, int pw, int lane) {
-    using C = Cfg<D>;
-    constexpr int CPR = D * 2 / 16;   // 16-byte chunks per row
-    constexpr int RPI = 32 / CPR;     // rows per warp instruction
-    constexpr int NI = 64 / RPI;      // warp instructions per producer warp
-    int ia = first + 64 * pw + lane, ib = ia + 32;
-    ia = ia < n_c ? ia : n_c - 1;
-    ib = ib < n_c ? ib : n_c - 1;
-    const int ra = rows(ia), rb = rows(ib);
-    const int c = lane % CPR;
-    const int rsub = lane / CPR;
-    const uint32_t box = static_cast<uint32_t>((c * 16) / C::SW);
-    const uint32_t cb = static_cast<uint32_t>(((c * 16) % C::SW) / 16);
-#pragma unroll
-    for (int k = 0; k < NI; ++k) {
-        const int rl = k * RPI + rsub;  // 0..63
-        const int grow = __shfl_sync(0xffffffffu, (k * RPI < 32) ? ra : rb, rl & 31);
-        const int r = 64 * pw + rl;     // tile row 0..127
-        const uint32_t sw = C::SW == 128 ? (cb ^ static_cast<uint32_t>(r & 7))
-                                         : (cb ^ static_cast<uint32_t>((r >> 1) & 3));
-        const uint32_t d = dst + box * C::BOX_BYTES + static_cast<uint32_t>(r) * C::SW + sw * 16u;
-        cp_async_16(d, g + static_cast<size_t>(grow) * D + c * 8);
-    }
-}
 
 template <int N>
 __device__ __forceinline__ float row_max(const uint32_t* v) {
@@ -533,7 +470,12 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             const int qi = q_first + qt * kBM + row;
             const float inv_l = 1.f / l_run;
             uint4* dst = nullptr;
-            if (qi < n_c) dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(rows(qi)) * D);
+            if (qi < n_c) {
+                const int grow = rows(qi);
+                dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(grow) * D);
+                // log-sum-exp (natural log) of the scaled scores: m*log2(e)/sqrt(d) + log2(l), in ln
+                if (p.lse) p.lse[grow] = (m_run * sl2 + ptx::lg2_approx(l_run)) * 0.6931471805599453f;
+            }
 #pragma unroll
             for (int g = 0; g < D / 32; ++g) {
                 uint32_t ov[32];

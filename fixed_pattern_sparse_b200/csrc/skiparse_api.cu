@@ -164,8 +164,25 @@ int skiparse_get_device_status(skiparse_stream_t stream) {
     return v;
 }
 
+static int attn_fwd_common(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int T, int H, int W, int heads, int d, int P, int mode,
+                           skiparse_stream_t stream);
+
 int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int T,
                         int H, int W, int heads, int d, int P, int mode, skiparse_stream_t stream) {
+    return attn_fwd_common(q, k, v, out, nullptr, B, T, H, W, heads, d, P, mode, stream);
+}
+
+int skiparse2d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int T, int H, int W, int heads, int d, int P, int mode,
+                            skiparse_stream_t stream) {
+    if (!lse) return SKIPARSE_ERR_INVALID_ARG;
+    return attn_fwd_common(q, k, v, out, lse, B, T, H, W, heads, d, P, mode, stream);
+}
+
+static int attn_fwd_common(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int T, int H, int W, int heads, int d, int P, int mode,
+                           skiparse_stream_t stream) {
     if (!q || !k || !v || !out) return SKIPARSE_ERR_INVALID_ARG;
     Geometry g;
     int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
@@ -175,11 +192,19 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     const size_t bytes = static_cast<size_t>(rows) * d * 2;
     if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
         return SKIPARSE_ERR_INVALID_ARG;
+    if (lse) {
+        if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return SKIPARSE_ERR_MISALIGNED;
+        const size_t lbytes = static_cast<size_t>(rows) * 4;
+        if (overlaps(lse, lbytes, q, bytes) || overlaps(lse, lbytes, k, bytes) ||
+            overlaps(lse, lbytes, v, bytes) || overlaps(lse, lbytes, out, bytes))
+            return SKIPARSE_ERR_INVALID_ARG;
+    }
     skiparse::AttnParams p{};
     p.q = static_cast<const uint16_t*>(q);
     p.k = static_cast<const uint16_t*>(k);
     p.v = static_cast<const uint16_t*>(v);
     p.out = static_cast<uint16_t*>(out);
+    p.lse = lse;
     p.status = status_ptr();
     if (!p.status) return SKIPARSE_ERR_CUDA;
     p.T = T; p.H = H; p.W = W; p.heads = heads; p.P = P; p.mode = mode;
@@ -191,6 +216,56 @@ int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.exchange(0);
     const int e = skiparse::launch_attn_fwd(p, g, stream);
+    return e == 0 ? SKIPARSE_OK : cuda_fail(e);
+}
+
+int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, float* delta,
+                        int B, int T, int H, int W, int heads, int d, int P, int mode,
+                        skiparse_stream_t stream) {
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return SKIPARSE_ERR_INVALID_ARG;
+    Geometry g;
+    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    if (st != SKIPARSE_OK) return st;
+    const void* bf[8] = {q, k, v, out, dout, dq, dk, dv};
+    for (const void* ptr : bf)
+        if (!aligned16(ptr)) return SKIPARSE_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(delta) & 3u))
+        return SKIPARSE_ERR_MISALIGNED;
+    const long long rows = static_cast<long long>(B) * T * H * W * heads;
+    const size_t tb = static_cast<size_t>(rows) * d * 2, vb = static_cast<size_t>(rows) * 4;
+    const void* outs[4] = {dq, dk, dv, delta};
+    const size_t out_bytes[4] = {tb, tb, tb, vb};
+    const void* ins[6] = {q, k, v, out, dout, lse};
+    const size_t in_bytes[6] = {tb, tb, tb, tb, tb, vb};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 6; ++j)
+            if (overlaps(outs[i], out_bytes[i], ins[j], in_bytes[j])) return SKIPARSE_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j])) return SKIPARSE_ERR_INVALID_ARG;
+    }
+    skiparse::BwdParams p{};
+    p.q = static_cast<const uint16_t*>(q);
+    p.k = static_cast<const uint16_t*>(k);
+    p.v = static_cast<const uint16_t*>(v);
+    p.out = static_cast<const uint16_t*>(out);
+    p.dout = static_cast<const uint16_t*>(dout);
+    p.lse = lse;
+    p.delta = delta;
+    p.dq = static_cast<uint16_t*>(dq);
+    p.dk = static_cast<uint16_t*>(dk);
+    p.dv = static_cast<uint16_t*>(dv);
+    p.status = status_ptr();
+    if (!p.status) return SKIPARSE_ERR_CUDA;
+    p.T = T; p.H = H; p.W = W; p.heads = heads; p.P = P; p.mode = mode;
+    for (int c = 0; c < skiparse::kMaxP; ++c) {
+        p.Rc[c] = g.Rc[c];
+        p.Sc[c] = g.Sc[c];
+    }
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    const int e = skiparse::launch_attn_bwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 

@@ -51,12 +51,33 @@ struct AttnParams {
     const uint16_t* k;
     const uint16_t* v;
     uint16_t* out;
+    float* lse;                    // optional (nullptr): log-sum-exp of q.k/sqrt(d) per (token, head)
     int* status;                   // device error word
     int T, H, W, heads, P, mode;
     int Rc[kMaxP], Sc[kMaxP];
     float scale_log2;              // log2(e)/sqrt(d)
     unsigned long long wait_limit_ns;
     int fault;                     // test hook: 1 = one producer never signals the first K tile
+};
+
+// Parameters of the backward kernels.
+struct BwdParams {
+    const uint16_t* q;             // bf16 bits, (B,T,H,W,heads,d)
+    const uint16_t* k;
+    const uint16_t* v;
+    const uint16_t* out;           // the forward output O
+    const uint16_t* dout;          // upstream gradient dO
+    const float* lse;              // (B,T,H,W,heads) natural-log log-sum-exp from the forward
+    float* delta;                  // (B,T,H,W,heads) D = rowsum(dO o O), written by the first launch
+    uint16_t* dq;
+    uint16_t* dk;
+    uint16_t* dv;
+    int* status;
+    int T, H, W, heads, P, mode;
+    int Rc[kMaxP], Sc[kMaxP];
+    float scale_log2;              // log2(e)/sqrt(d)
+    float scale;                   // 1/sqrt(d)
+    unsigned long long wait_limit_ns;
 };
 
 struct RearrangeParams {
@@ -73,6 +94,7 @@ enum : int { kOk = 0, kErrTimeout = 5 };
 
 // Launchers (defined in the kernel translation units). They return the cudaError_t as int.
 int launch_attn_fwd(const AttnParams& p, const Geometry& g, void* stream);
+int launch_attn_bwd(const BwdParams& p, const Geometry& g, void* stream);
 int launch_rearrange(const RearrangeParams& p, int kind, void* stream);  // 0 fwd, 1 inverse, 2 switch
 int attn_smem_bytes(int d);
 int launch_exp2(const float* x, float* y, long long n, int method, void* stream);

@@ -74,6 +74,34 @@ SKIPARSE_API int skiparse2d_attn_fwd(const void* q, const void* k, const void* v
                         skiparse_stream_t stream);
 
 /*
+ * Forward as skiparse2d_attn_fwd that also writes, for the backward pass,
+ *   lse : (B, T, H, W, heads) fp32, 4-byte aligned, written for every real token:
+ *         lse[x] = log sum_y exp(q[x].k[y] / sqrt(d)) over the keys y of x's class (natural log).
+ * lse must not overlap q, k, v or out.
+ */
+SKIPARSE_API int skiparse2d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out,
+                                         float* lse, int B, int T, int H, int W, int heads, int d,
+                                         int P, int mode, skiparse_stream_t stream);
+
+/*
+ * Backward pass of skiparse2d_attn_fwd (for fine-tuning the sparse model). With, inside each
+ * class subsequence, P = softmax(q.k^T/sqrt(d)) and D_x = dout[x].out[x]:
+ *   dv = P^T dout,  dS = P o (dout v^T - D),  dq = dS k / sqrt(d),  dk = dS^T q / sqrt(d).
+ *   q, k, v, out, dout : (B, T, H, W, heads, d) bf16, read-only; out is the forward's output.
+ *   lse                : (B, T, H, W, heads) fp32 from skiparse2d_attn_fwd_lse, read-only.
+ *   dq, dk, dv         : (B, T, H, W, heads, d) bf16, written entirely.
+ *   delta              : (B, T, H, W, heads) fp32 workspace owned by the caller; on return it
+ *                        holds D. 4-byte aligned.
+ * None of dq, dk, dv, delta may overlap each other or an input. Three kernel launches (D, then
+ * the key-tile-major dk/dv kernel, then the query-tile-major dq kernel); no atomics, results
+ * are deterministic.
+ */
+SKIPARSE_API int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                     const void* dout, const float* lse, void* dq, void* dk,
+                                     void* dv, float* delta, int B, int T, int H, int W, int heads,
+                                     int d, int P, int mode, skiparse_stream_t stream);
+
+/*
  * Rearrange (方法步骤详情: the rearrange that forms the P^2 subsequences, with padding).
  *   x : (B, T, H, W, heads, d) bf16, read-only.
  *   y : (B*P*P, n, heads, d) bf16, skiparse_rearranged_numel() elements, written entirely;

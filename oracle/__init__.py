@@ -14,6 +14,9 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
       invariants, two-hop property);
   switch_mode -- pinned (equals unrearrange of one mode followed by rearrange of the other;
       a switch there and back is the identity on real slots; pads are zero);
+  attn_bwd, attn_bwd_rows -- pinned (torch autograd through an independent dense masked fp64
+      attention; P=1 against autograd of fp64 scaled_dot_product_attention; central finite
+      differences of the forward oracle; sampled rows equal the full result);
   attn_fwd, attn_fwd_rows, masked_attention -- pinned (P=1 against fp64
       scaled_dot_product_attention, numpy brute force with an explicit 2-D mask,
       closed forms, pad invariance).
@@ -61,6 +64,10 @@ def lib():
         L.oracle_attn_fwd.restype = c_int
         L.oracle_attn_fwd_rows.argtypes = [vp, vp, vp, vp, c_ll, vp] + shape8 + [c_int]
         L.oracle_attn_fwd_rows.restype = c_int
+        L.oracle_attn_bwd.argtypes = [vp] * 8 + shape8 + [c_int]
+        L.oracle_attn_bwd.restype = c_int
+        L.oracle_attn_bwd_rows.argtypes = [vp, vp, vp, vp, vp, c_ll, vp, vp, vp] + shape8 + [c_int]
+        L.oracle_attn_bwd_rows.restype = c_int
         _LIB = L
     return _LIB
 
@@ -177,3 +184,28 @@ def attn_fwd_rows(q, k, v, rows, P: int, mode: int, nthreads: int | None = None)
                                       _ptr(out), B, T, H, W, heads, d, P, mode,
                                       nthreads or default_threads()), "attn_fwd_rows")
     return out
+
+
+def attn_bwd(q, k, v, dout, P: int, mode: int, nthreads: int | None = None):
+    """Backward pass in fp64: returns (dq, dk, dv, lse); lse is the natural-log log-sum-exp of
+    q.k/sqrt(d) over each token's class, shape (B,T,H,W,heads)."""
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, T, H, W, heads, d = qb.shape
+    dq, dk, dv = (np.empty(qb.shape, dtype=np.float64) for _ in range(3))
+    lse = np.empty((B, T, H, W, heads), dtype=np.float64)
+    _check(lib().oracle_attn_bwd(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(lse), B, T, H, W, heads, d, P, mode, nthreads or default_threads()),
+           "attn_bwd")
+    return dq, dk, dv, lse
+
+
+def attn_bwd_rows(q, k, v, dout, rows, P: int, mode: int, nthreads: int | None = None):
+    """Backward for selected rows (token*heads + head): (dq, dk, dv), each (nrows, d) fp64."""
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, T, H, W, heads, d = qb.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    dq, dk, dv = (np.zeros((rows.shape[0], d), dtype=np.float64) for _ in range(3))
+    _check(lib().oracle_attn_bwd_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(gb), _ptr(rows), rows.shape[0],
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, T, H, W, heads, d, P, mode,
+                                      nthreads or default_threads()), "attn_bwd_rows")
+    return dq, dk, dv

@@ -56,3 +56,41 @@ def attention(q, k, v, P: int, mode: int) -> np.ndarray:
             O[real] = A @ V
             out[b, ..., hd, :] = O.reshape(T, Hp, Wp, d)
     return out[:, :, :H, :W]
+
+
+def attention_torch(q, k, v, P: int, mode: int):
+    """The same dense masked attention in torch fp64, differentiable (autograd gives the
+    backward pass of the definition). Returns (out, lse) with lse the natural-log
+    log-sum-exp of q.k/sqrt(d) over each real query's allowed keys."""
+    import torch
+    B, T, H, W, heads, d = q.shape
+    step = P * P
+    Hp = -(-H // step) * step
+    Wp = -(-W // step) * step
+    pad = (0, 0, 0, 0, 0, Wp - W, 0, Hp - H)
+    qp, kp, vp = (torch.nn.functional.pad(a, pad) for a in (q, k, v))
+    cls = torch.from_numpy(np.broadcast_to(class_grid(Hp, Wp, P, mode), (T, Hp, Wp)).reshape(-1).copy())
+    real = torch.zeros((T, Hp, Wp), dtype=torch.bool)
+    real[:, :H, :W] = True
+    real = real.reshape(-1)
+    mask = (cls[:, None] == cls[None, :]) & real[None, :]
+    N = T * Hp * Wp
+    outs, lses = [], []
+    for b in range(B):
+        ob, lb = [], []
+        for hd in range(heads):
+            Q = qp[b, ..., hd, :].reshape(N, d)[real]
+            K = kp[b, ..., hd, :].reshape(N, d)
+            V = vp[b, ..., hd, :].reshape(N, d)
+            S = (Q @ K.T) / (d ** 0.5)
+            S = S.masked_fill(~mask[real], float("-inf"))
+            lse = torch.logsumexp(S, dim=1)
+            A = torch.exp(S - lse[:, None])
+            ob.append(A @ V)
+            lb.append(lse)
+        outs.append(torch.stack(ob, dim=1))   # (Nreal, heads, d)
+        lses.append(torch.stack(lb, dim=1))   # (Nreal, heads)
+    out = torch.stack(outs)                    # (B, Nreal, heads, d)
+    lse = torch.stack(lses)
+    # back to (B, T, H, W, heads, ...): real tokens in (t, h, w) order are exactly [:, :, :H, :W]
+    return out.reshape(B, T, H, W, heads, d), lse.reshape(B, T, H, W, heads)

@@ -460,3 +460,322 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
     free(key); free(sq); free(sk); free(sv); free(valid); free(pos); free(slot); free(th); free(jobs);
     return rc;
 }
+
+
+/* ------------------------------------------------------------------ backward pass
+ * Gradients of the Skiparse-2D forward for an upstream gradient dO, by the definition of
+ * softmax attention inside each subsequence (the same three steps as the forward: rearrange
+ * with the pad mask, per-subsequence dense attention -- here its derivative -- and rearrange
+ * back). With s_ij = q_i.k_j, L_i = log sum_j exp(s_ij/sqrt(d)), P_ij = exp(s_ij/sqrt(d) - L_i),
+ * O_i = sum_j P_ij v_j, D_i = dO_i.O_i:
+ *   dV_j = sum_i P_ij dO_i,  dP_ij = dO_i.v_j,  dS_ij = P_ij (dP_ij - D_i),
+ *   dQ_i = sum_j dS_ij k_j / sqrt(d),  dK_j = sum_i dS_ij q_i / sqrt(d).               */
+
+typedef struct {
+    const uint16_t *yq, *yk, *yv, *ydo;
+    const uint8_t* valid;
+    double *ydq, *ydk, *ydv, *ylse;   /* (nseq, n, heads, d) / (nseq, n, heads) */
+    long long nseq, n;
+    int heads, d;
+    int tid, nthreads;
+} bwd_job;
+
+static void* bwd_worker(void* arg) {
+    bwd_job* jb = (bwd_job*)arg;
+    const long long n = jb->n;
+    const int d = jb->d, heads = jb->heads;
+    const long long row = (long long)heads * d;
+    const double scale = 1.0 / sqrt((double)d);
+    double* p = (double*)malloc(sizeof(double) * (size_t)n);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!p || !dp || !o) { free(p); free(dp); free(o); return (void*)1; }
+    for (long long unit = jb->tid; unit < jb->nseq * heads; unit += jb->nthreads) {
+        const long long seq = unit / heads;
+        const int head = (int)(unit % heads);
+        #define AT(buf, j) ((buf) + (seq * n + (j)) * row + (long long)head * d)
+        for (long long i = 0; i < n; ++i) {
+            if (!jb->valid[seq * n + i]) continue;
+            const uint16_t* qi = AT(jb->yq, i);
+            const uint16_t* doi = AT(jb->ydo, i);
+            double m = -INFINITY;
+            for (long long j = 0; j < n; ++j) {
+                if (!jb->valid[seq * n + j]) continue;
+                const uint16_t* kj = AT(jb->yk, j);
+                double acc = 0.0;
+                for (int e = 0; e < d; ++e) acc += bf16_bits_to_double(qi[e]) * bf16_bits_to_double(kj[e]);
+                p[j] = acc * scale;
+                if (p[j] > m) m = p[j];
+            }
+            double sum = 0.0;
+            for (long long j = 0; j < n; ++j)
+                if (jb->valid[seq * n + j]) sum += exp(p[j] - m);
+            const double lse = m + log(sum);
+            if (jb->ylse) jb->ylse[(seq * n + i) * heads + head] = lse;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (long long j = 0; j < n; ++j) {
+                if (!jb->valid[seq * n + j]) continue;
+                p[j] = exp(p[j] - lse);
+                const uint16_t* vj = AT(jb->yv, j);
+                for (int e = 0; e < d; ++e) o[e] += p[j] * bf16_bits_to_double(vj[e]);
+            }
+            double D = 0.0;
+            for (int e = 0; e < d; ++e) D += bf16_bits_to_double(doi[e]) * o[e];
+            double* dqi = jb->ydq + (seq * n + i) * row + (long long)head * d;
+            for (long long j = 0; j < n; ++j) {
+                if (!jb->valid[seq * n + j]) continue;
+                const uint16_t* vj = AT(jb->yv, j);
+                const uint16_t* kj = AT(jb->yk, j);
+                double dpv = 0.0;
+                for (int e = 0; e < d; ++e) dpv += bf16_bits_to_double(doi[e]) * bf16_bits_to_double(vj[e]);
+                const double ds = p[j] * (dpv - D);
+                double* dvj = jb->ydv + (seq * n + j) * row + (long long)head * d;
+                double* dkj = jb->ydk + (seq * n + j) * row + (long long)head * d;
+                for (int e = 0; e < d; ++e) {
+                    dvj[e] += p[j] * bf16_bits_to_double(doi[e]);
+                    dkj[e] += ds * bf16_bits_to_double(qi[e]) * scale;
+                    dqi[e] += ds * bf16_bits_to_double(kj[e]) * scale;
+                }
+            }
+        }
+        #undef AT
+    }
+    free(p); free(dp); free(o);
+    return NULL;
+}
+
+int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                    double* dq, double* dk, double* dv, double* lse,
+                    int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads) {
+    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+    if (nthreads < 1) nthreads = 1;
+    rearranged r;
+    long long n = 0;
+    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
+    if (rc) return rc;
+    const long long nseq = (long long)B * P * P;
+    const size_t elems = (size_t)(nseq * n * heads * d);
+    uint16_t* ydo = (uint16_t*)malloc(elems * 2);
+    double* ydq = (double*)calloc(elems, sizeof(double));
+    double* ydk = (double*)calloc(elems, sizeof(double));
+    double* ydv = (double*)calloc(elems, sizeof(double));
+    double* ylse = lse ? (double*)calloc((size_t)(nseq * n * heads), sizeof(double)) : NULL;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    bwd_job* jobs = (bwd_job*)malloc(sizeof(bwd_job) * (size_t)nthreads);
+    if (!ydo || !ydq || !ydk || !ydv || (lse && !ylse) || !th || !jobs) rc = -2;
+    if (!rc) {
+        oracle_rearrange(dout, ydo, NULL, B, T, H, W, heads, d, P, mode);
+        int started = 0;
+        for (int t = 0; t < nthreads; ++t) {
+            bwd_job* jb = &jobs[t];
+            jb->yq = r.yq; jb->yk = r.yk; jb->yv = r.yv; jb->ydo = ydo; jb->valid = r.valid;
+            jb->ydq = ydq; jb->ydk = ydk; jb->ydv = ydv; jb->ylse = ylse;
+            jb->nseq = nseq; jb->n = n; jb->heads = heads; jb->d = d;
+            jb->tid = t; jb->nthreads = nthreads;
+            if (pthread_create(&th[t], NULL, bwd_worker, jb) != 0) { rc = -3; break; }
+            ++started;
+        }
+        for (int t = 0; t < started; ++t) {
+            void* ret = NULL;
+            pthread_join(th[t], &ret);
+            if (ret) rc = -2;
+        }
+    }
+    if (!rc) {
+        oracle_unrearrange_f64(ydq, dq, B, T, H, W, heads, d, P, mode);
+        oracle_unrearrange_f64(ydk, dk, B, T, H, W, heads, d, P, mode);
+        oracle_unrearrange_f64(ydv, dv, B, T, H, W, heads, d, P, mode);
+        if (lse) oracle_unrearrange_f64(ylse, lse, B, T, H, W, heads, 1, P, mode);
+    }
+    free(ydo); free(ydq); free(ydk); free(ydv); free(ylse); free(th); free(jobs);
+    free_rearranged(&r);
+    return rc;
+}
+
+/* Gradients for selected rows (token*heads + head of the original layout): dq of the token as
+ * a query, dk and dv of the token as a key. Per (subsequence, head) holding a requested row:
+ * the subsequence is gathered as in oracle_attn_fwd_rows, L_i and D_i are computed for all of
+ * its queries, then each requested row's gradients follow from the formulas above. */
+typedef struct {
+    const uint16_t *sq, *sk, *sv, *sdo;   /* one subsequence, one head: (n, d) */
+    const uint8_t* valid;
+    long long n;
+    int d;
+    double *L, *Dl;                       /* (n) */
+    const long long* pos; const long long* slot; long long count;
+    double *dq, *dk, *dv;                 /* requested rows (nrows, d) */
+    int phase;                            /* 0: L and D for every query; 1: requested rows */
+    int tid, nthreads;
+} bwdrows_job;
+
+static double dotbf(const uint16_t* a, const uint16_t* b, int d) {
+    double acc = 0.0;
+    for (int e = 0; e < d; ++e) acc += bf16_bits_to_double(a[e]) * bf16_bits_to_double(b[e]);
+    return acc;
+}
+
+static void* bwdrows_worker(void* arg) {
+    bwdrows_job* jb = (bwdrows_job*)arg;
+    const long long n = jb->n;
+    const int d = jb->d;
+    const double scale = 1.0 / sqrt((double)d);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    double* sc = (double*)malloc(sizeof(double) * (size_t)n);
+    if (!o || !sc) { free(o); free(sc); return (void*)1; }
+    if (jb->phase == 0) {
+        for (long long i = jb->tid; i < n; i += jb->nthreads) {
+            if (!jb->valid[i]) continue;
+            double m = -INFINITY;
+            for (long long j = 0; j < n; ++j) {
+                if (!jb->valid[j]) continue;
+                sc[j] = dotbf(jb->sq + i * d, jb->sk + j * d, d) * scale;
+                if (sc[j] > m) m = sc[j];
+            }
+            double sum = 0.0;
+            for (long long j = 0; j < n; ++j) if (jb->valid[j]) sum += exp(sc[j] - m);
+            const double L = m + log(sum);
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (long long j = 0; j < n; ++j) {
+                if (!jb->valid[j]) continue;
+                const double pij = exp(sc[j] - L);
+                for (int e = 0; e < d; ++e) o[e] += pij * bf16_bits_to_double(jb->sv[j * d + e]);
+            }
+            double D = 0.0;
+            for (int e = 0; e < d; ++e) D += bf16_bits_to_double(jb->sdo[i * d + e]) * o[e];
+            jb->L[i] = L;
+            jb->Dl[i] = D;
+        }
+    } else {
+        for (long long u = jb->tid; u < jb->count; u += jb->nthreads) {
+            const long long x = jb->pos[u];
+            double* dq = jb->dq + jb->slot[u] * (long long)d;
+            double* dk = jb->dk + jb->slot[u] * (long long)d;
+            double* dv = jb->dv + jb->slot[u] * (long long)d;
+            for (int e = 0; e < d; ++e) { dq[e] = 0.0; dk[e] = 0.0; dv[e] = 0.0; }
+            if (!jb->valid[x]) continue;
+            for (long long j = 0; j < n; ++j) {          /* x as the query */
+                if (!jb->valid[j]) continue;
+                const double pxj = exp(dotbf(jb->sq + x * d, jb->sk + j * d, d) * scale - jb->L[x]);
+                const double ds = pxj * (dotbf(jb->sdo + x * d, jb->sv + j * d, d) - jb->Dl[x]);
+                for (int e = 0; e < d; ++e) dq[e] += ds * bf16_bits_to_double(jb->sk[j * d + e]) * scale;
+            }
+            for (long long i = 0; i < n; ++i) {          /* x as the key */
+                if (!jb->valid[i]) continue;
+                const double pix = exp(dotbf(jb->sq + i * d, jb->sk + x * d, d) * scale - jb->L[i]);
+                const double ds = pix * (dotbf(jb->sdo + i * d, jb->sv + x * d, d) - jb->Dl[i]);
+                for (int e = 0; e < d; ++e) {
+                    dk[e] += ds * bf16_bits_to_double(jb->sq[i * d + e]) * scale;
+                    dv[e] += pix * bf16_bits_to_double(jb->sdo[i * d + e]);
+                }
+            }
+        }
+    }
+    free(o); free(sc);
+    return NULL;
+}
+
+static int run_bwdrows(bwdrows_job proto, int nthreads, int phase) {
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    bwdrows_job* jobs = (bwdrows_job*)malloc(sizeof(bwdrows_job) * (size_t)nthreads);
+    int rc = 0, started = 0;
+    if (!th || !jobs) { free(th); free(jobs); return -2; }
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = proto;
+        jobs[t].phase = phase; jobs[t].tid = t; jobs[t].nthreads = nthreads;
+        if (pthread_create(&th[t], NULL, bwdrows_worker, &jobs[t]) != 0) { rc = -3; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) {
+        void* ret = NULL;
+        pthread_join(th[t], &ret);
+        if (ret) rc = -2;
+    }
+    free(th); free(jobs);
+    return rc;
+}
+
+int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                         const long long* rows, long long nrows, double* dq_rows, double* dk_rows,
+                         double* dv_rows, int B, int T, int H, int W, int heads, int d, int P,
+                         int mode, int nthreads) {
+    if (check_shape(B, T, H, W, heads, d, P, mode) || nrows < 0) return -1;
+    const long long ntok = (long long)B * T * H * W;
+    for (long long i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= ntok * heads) return -1;
+    if (nrows == 0) return 0;
+    if (nthreads < 1) nthreads = 1;
+    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
+    const int R = Hp / P, S = Wp / P;
+    const long long n = (long long)T * R * S;
+    const long long q2 = (long long)P * P;
+    long long* key = (long long*)malloc(sizeof(long long) * (size_t)nrows * 2);
+    if (!key) return -2;
+    for (long long i = 0; i < nrows; ++i) {
+        const int head = (int)(rows[i] % heads);
+        long long tok = rows[i] / heads;
+        const int w = (int)(tok % W); tok /= W;
+        const int h = (int)(tok % H); tok /= H;
+        const int t = (int)(tok % T);
+        const int b = (int)(tok / T);
+        int ci, rr, cj, ss;
+        oracle_axis_map(h, P, mode, &ci, &rr);
+        oracle_axis_map(w, P, mode, &cj, &ss);
+        const long long seq = (long long)b * q2 + ci * P + cj;
+        key[2 * i] = (seq * heads + head) * n + ((long long)t * R + rr) * S + ss;
+        key[2 * i + 1] = i;
+    }
+    qsort(key, (size_t)nrows, 2 * sizeof(long long), cmp_ll);
+    uint16_t* sq = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint16_t* sk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint16_t* sv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint16_t* sdo = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
+    uint8_t* valid = (uint8_t*)malloc((size_t)n);
+    double* L = (double*)malloc(sizeof(double) * (size_t)n);
+    double* Dl = (double*)malloc(sizeof(double) * (size_t)n);
+    long long* pos = (long long*)malloc(sizeof(long long) * (size_t)nrows);
+    long long* slot = (long long*)malloc(sizeof(long long) * (size_t)nrows);
+    int rc = 0;
+    if (!sq || !sk || !sv || !sdo || !valid || !L || !Dl || !pos || !slot) rc = -2;
+    for (long long g0 = 0; rc == 0 && g0 < nrows;) {
+        const long long group = key[2 * g0] / n;
+        long long g1 = g0;
+        while (g1 < nrows && key[2 * g1] / n == group) {
+            pos[g1 - g0] = key[2 * g1] % n;
+            slot[g1 - g0] = key[2 * g1 + 1];
+            ++g1;
+        }
+        const long long seq = group / heads;
+        const int head = (int)(group % heads);
+        const int b = (int)(seq / q2);
+        const int c = (int)(seq % q2);
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hp; ++h)
+                for (int w = 0; w < Wp; ++w) {
+                    int ci, rr, cj, ss;
+                    oracle_axis_map(h, P, mode, &ci, &rr);
+                    oracle_axis_map(w, P, mode, &cj, &ss);
+                    if (ci * P + cj != c) continue;
+                    const long long pp = ((long long)t * R + rr) * S + ss;
+                    const int real = (h < H) && (w < W);
+                    valid[pp] = (uint8_t)real;
+                    const long long src = ((((long long)b * T + t) * H + h) * W + w) * heads + head;
+                    for (int e = 0; e < d; ++e) {
+                        sq[pp * d + e] = real ? q[src * d + e] : 0;
+                        sk[pp * d + e] = real ? k[src * d + e] : 0;
+                        sv[pp * d + e] = real ? v[src * d + e] : 0;
+                        sdo[pp * d + e] = real ? dout[src * d + e] : 0;
+                    }
+                }
+        bwdrows_job jb;
+        memset(&jb, 0, sizeof jb);
+        jb.sq = sq; jb.sk = sk; jb.sv = sv; jb.sdo = sdo; jb.valid = valid;
+        jb.n = n; jb.d = d; jb.L = L; jb.Dl = Dl;
+        jb.pos = pos; jb.slot = slot; jb.count = g1 - g0;
+        jb.dq = dq_rows; jb.dk = dk_rows; jb.dv = dv_rows;
+        rc = run_bwdrows(jb, nthreads, 0);
+        if (!rc) rc = run_bwdrows(jb, nthreads, 1);
+        g0 = g1;
+    }
+    free(key); free(sq); free(sk); free(sv); free(sdo); free(valid); free(L); free(Dl); free(pos); free(slot);
+    return rc;
+}

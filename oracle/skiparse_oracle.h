@@ -70,6 +70,20 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
                          int B, int T, int H, int W, int heads, int d, int P, int mode,
                          int nthreads);
 
+/* Backward pass for an upstream gradient dout (all (B,T,H,W,heads,d) bf16 bits): dq, dk, dv
+ * (B,T,H,W,heads,d) fp64; lse (B,T,H,W,heads) fp64, natural-log log-sum-exp of q.k/sqrt(d)
+ * over each token's class (may be NULL). */
+int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                    double* dq, double* dk, double* dv, double* lse,
+                    int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads);
+
+/* Backward for selected rows (token*heads + head): dq of the token as a query, dk and dv of
+ * the token as a key; each output (nrows, d) fp64. */
+int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                         const long long* rows, long long nrows, double* dq_rows, double* dk_rows,
+                         double* dv_rows, int B, int T, int H, int W, int heads, int d, int P,
+                         int mode, int nthreads);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,3 +67,14 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
     bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
     assert capsys.readouterr().out == ""
+
+
+def test_hybrid_stack_schedule():
+    """4 dense blocks at each end, alternating sparse modes in between (the pages' hybrid)."""
+    import bench
+    sched = bench.stack_schedule(40, 4, 4)
+    assert len(sched) == 40
+    assert all(p == 1 for p, _ in sched[:4] + sched[-4:])
+    middle = sched[4:-4]
+    assert all(p is None for p, _ in middle) and len(middle) == 32
+    assert [m for _, m in middle] == [0, 1] * 16
