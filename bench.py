@@ -340,6 +340,39 @@ def run_ours(args):
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the dense comparison")
 
+    # backward pass (fine-tuning): 3 launches per call, FLOPs counted as 2.5x the forward's
+    # (dV, dP, dQ, dK and the recomputed S: the standard accounting of attention backward)
+    bwd = None
+    if not args.no_backward:
+        gd = synth.randn_bf16(w.shape, 1000 * w.family + 7).to(dev)
+        outs, lses = [], []
+        for m in modes:
+            o_m, l_m = fps.skiparse2d_attn_fwd_lse(qd, kd, vd, w.P, m)
+            outs.append(o_m)
+            lses.append(l_m)
+        dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+        delta = torch.empty(qd.shape[:5], dtype=torch.float32, device=dev)
+
+        def bstep(i):
+            j = i % len(modes)
+            fps.skiparse2d_attn_bwd(qd, kd, vd, outs[j], gd, lses[j], w.P, modes[j], dq=dq, dk=dk, dv=dv, delta=delta)
+
+        for i in range(3):
+            bstep(i)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for i in range(args.backward_steps):
+            bstep(i)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = b0.elapsed_time(b1) / args.backward_steps
+        if fps.get_device_status() != 0:
+            raise SystemExit("device status error in the backward timing")
+        bwd = {"ms_per_call": round(bms, 3), "tflops": round(2.5 * fl / (bms / 1e3) / 1e12, 1),
+               "flop_formula": "2.5 x the forward's padded-formula FLOPs",
+               "launches_per_call": 3, "forward_plus_backward_ms": round(bms + statistics.mean(per_launch), 3)}
+        del gd, outs, lses, dq, dk, dv, delta
+
     # standalone rearrange / unrearrange bandwidth (HBM-bound permutation of token rows)
     rearr = None
     if not args.no_rearrange:
@@ -402,6 +435,7 @@ def run_ours(args):
             "tflops_real_pairs": real,
             "dense_p1": dense,
             "rearrange_kernels": rearr,
+            "backward": bwd,
             "kernel_hash": kernel_hash(),
         }
         print(json.dumps(line), flush=True)
@@ -545,6 +579,8 @@ def main(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rearrange", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-steps", type=int, default=4)
     ap.add_argument("--rearrange-steps", type=int, default=10)
     ap.add_argument("--stack", action="store_true",
                     help="time a hybrid stack of dense and alternating Skiparse-2D layers instead")

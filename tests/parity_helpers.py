@@ -42,3 +42,18 @@ def check_close(got: np.ndarray, want: np.ndarray, what: str):
     mx, mean = float(err.max()), float(err.mean())
     assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max|err|={mx:.3e} mean|err|={mean:.3e}"
     return mx, mean
+
+
+def sample_rows_one_class(w, mode: int, count: int, cls: int = 0, head: int = 0, seed: int = 0) -> np.ndarray:
+    """Rows (token*heads + head) of one (class, head) subsequence of batch element 0: its first
+    and last real tokens plus `count` random ones (class rule from the brute force's own
+    restatement). One subsequence keeps the backward oracle's per-subsequence cost bounded."""
+    from oracle import brute
+    step = w.P * w.P
+    Hp, Wp = -(-w.H // step) * step, -(-w.W // step) * step
+    grid = brute.class_grid(Hp, Wp, w.P, mode)[: w.H, : w.W]
+    hh, ww = np.nonzero(grid == cls)
+    toks = (np.arange(w.T)[:, None] * w.H * w.W + (hh * w.W + ww)[None, :]).reshape(-1)
+    rng = np.random.default_rng(seed)
+    pick = np.unique(np.concatenate([toks[:2], toks[-2:], rng.choice(toks, size=min(count, len(toks)), replace=False)]))
+    return pick.astype(np.int64) * w.heads + head

@@ -3,8 +3,10 @@
 Tolerance (derived in the design notes from the arithmetic): the kernels round P and dS to
 bf16 before their tensor-core products and round the gradients to bf16 once; relative to the
 largest gradient entry that gives errors of a few bf16 half-ulps (2^-9). We require
-max|err| <= 2e-2 * max|ref| and mean|err| <= 2e-3 * max|ref| for each of dq, dk, dv, and the
-forward's lse within 1e-3 absolute."""
+max|err| <= 2e-2 * max|ref| and mean|err| <= 2e-3 * max|ref| for each of dq, dk, dv (max|ref|
+floored at 1e-3 for gradients that are exactly zero), and the forward's lse within 1e-3.
+Full-size shapes are checked on sampled rows of one (class, head) subsequence, the last class
+and head (ragged in the padded workloads)."""
 
 from __future__ import annotations
 
@@ -14,7 +16,7 @@ import torch
 
 import oracle
 import skiparse_synth as synth
-from parity_helpers import sample_rows
+from parity_helpers import sample_rows_one_class
 
 pytestmark = pytest.mark.gpu
 TOK, GRP = 0, 1
@@ -31,7 +33,7 @@ def fps():
 def check_grad(got, want, what):
     got = np.asarray(got, dtype=np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite"
-    scale = max(np.abs(want).max(), 1e-30)
+    scale = max(np.abs(want).max(), 1e-3)  # exact zeros (e.g. a single-token class's dq) need a floor
     err = np.abs(got - want)
     print(f"{what}: max|err|/max|ref| = {err.max() / scale:.3e}, mean|err|/max|ref| = {err.mean() / scale:.3e}")
     assert err.max() <= 2e-2 * scale and err.mean() <= 2e-3 * scale, what
@@ -68,7 +70,7 @@ def test_backward_full_size_sampled(fps, name, mode):
     out, lse = fps.skiparse2d_attn_fwd_lse(qd, kd, vd, w.P, mode)
     dq, dk, dv = fps.skiparse2d_attn_bwd(qd, kd, vd, out, gd, lse, w.P, mode)
     assert fps.get_device_status() == 0
-    rows = sample_rows(w, 24, seed=w.family)
+    rows = sample_rows_one_class(w, mode, 24, cls=w.P * w.P - 1, head=w.heads - 1, seed=w.family)
     rq, rk, rv = oracle.attn_bwd_rows(q, k, v, dout, rows, w.P, mode)
     idx = torch.from_numpy(rows).cuda()
     for got, want, what in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
