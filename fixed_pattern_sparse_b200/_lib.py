@@ -18,6 +18,7 @@ SIGNATURES = {
     "skiparse2d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse2d_attn_fwd_lse": (_I, [_VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse2d_attn_bwd": (_I, [_VP] * 10 + [_I] * 8 + [_VP]),
+    "skiparse2d_attn_bwd_noalloc": (_I, [_VP] * 9 + [_I] * 8 + [_VP]),
     "skiparse_rearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_unrearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse_switch_mode": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),

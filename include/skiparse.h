@@ -102,6 +102,28 @@ SKIPARSE_API int skiparse2d_attn_bwd(const void* q, const void* k, const void* v
                                      int d, int P, int mode, skiparse_stream_t stream);
 
 /*
+ * Backward pass for callers that cannot allocate device memory (the pages have no counterpart:
+ * this is an interface convenience). Same arguments, kernels and results as skiparse2d_attn_bwd
+ * without `delta`: the D workspace lives in a fixed array owned by the library instead -- 2^22
+ * fp32 values (16 MiB) that every device loading the library holds until the process exits.
+ * For callers whose host framework owns all device memory, or that must not call the allocator.
+ *   - B*T*H*W*heads must be at most 4,194,304; larger problems get SKIPARSE_ERR_UNSUPPORTED
+ *     before anything is launched (use skiparse2d_attn_bwd with your own workspace instead).
+ *   - Allocates nothing: no cudaMalloc or cudaFree, no allocating library call.
+ *   - The first call on a device looks up the workspace's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that first call
+ *     before any stream capture.
+ *   - All calls share the one workspace per device: calls that can run at the same time on
+ *     the GPU (on different streams) race on it and must be ordered by the caller. The
+ *     previous call's contents never matter; nothing needs clearing between calls.
+ */
+SKIPARSE_API int skiparse2d_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                             const void* out, const void* dout, const float* lse,
+                                             void* dq, void* dk, void* dv, int B, int T, int H,
+                                             int W, int heads, int d, int P, int mode,
+                                             skiparse_stream_t stream);
+
+/*
  * Rearrange (方法步骤详情: the rearrange that forms the P^2 subsequences, with padding).
  *   x : (B, T, H, W, heads, d) bf16, read-only.
  *   y : (B*P*P, n, heads, d) bf16, skiparse_rearranged_numel() elements, written entirely;
