@@ -50,8 +50,8 @@ constexpr int kBN = 128;   // keys per tile
 #endif
 constexpr int kThreads = SKIPARSE_REGSPLIT ? 384 : 352;
 constexpr int kLaunchRegs = 168;       // 65536 / 384 rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 216;      // 2 x 128 x 216 + 128 x 64 <= 384 x 168
-constexpr int kOtherRegs = 64;
+[[maybe_unused]] constexpr int kSoftmaxRegs = 216;  // 2 x 128 x 216 + 128 x 64 <= 384 x 168
+[[maybe_unused]] constexpr int kOtherRegs = 64;
 constexpr int kProdWarp0 = 8;
 constexpr int kNumProducers = 64;
 constexpr int kMmaWarp = 10;
