@@ -94,3 +94,89 @@ def attention_torch(q, k, v, P: int, mode: int):
     lse = torch.stack(lses)
     # back to (B, T, H, W, heads, ...): real tokens in (t, h, w) order are exactly [:, :, :H, :W]
     return out.reshape(B, T, H, W, heads, d), lse.reshape(B, T, H, W, heads)
+
+
+# ---------------------------------------------------------------------------- Skiparse-1D
+# The 1D skip pattern on the flattened sequence (the variant the summary page's 技术新颖性 and
+# 实验结果 sections compare Skiparse-2D with). Reading: the flattened in-frame index
+# x = h*W + w, ratio k = P^2; token-wise class x mod k, group-wise class (x div k) mod k; each
+# frame's H*W positions padded at the end to a multiple of k^2. Written here from that reading,
+# separately from the C oracle.
+
+def class_1d(Lp: int, P: int, mode: int) -> np.ndarray:
+    x = np.arange(Lp)
+    k = P * P
+    return (x % k if mode == 0 else (x // k) % k).astype(np.int64)
+
+
+def _frames_1d(a, P: int):
+    """(B,T,H,W,heads,d) -> (B, T, Lp, heads, d) with the in-frame index flattened and padded."""
+    B, T, H, W, heads, d = a.shape
+    k2 = (P * P) ** 2
+    L = H * W
+    Lp = -(-L // k2) * k2
+    flat = a.reshape(B, T, L, heads, d)
+    return flat, L, Lp
+
+
+def attention_1d(q, k, v, P: int, mode: int) -> np.ndarray:
+    """Skiparse-1D forward by one dense fp64 attention per (batch, head) over all padded
+    positions of all frames with the mask [class(x) == class(y)] and [y real]."""
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, T, H, W, heads, d = q.shape
+    (qf, L, Lp), (kf, _, _), (vf, _, _) = (_frames_1d(a, P) for a in (q, k, v))
+    pad = ((0, 0), (0, 0), (0, Lp - L), (0, 0), (0, 0))
+    qp, kp, vp = (np.pad(a, pad) for a in (qf, kf, vf))
+    cls = np.broadcast_to(class_1d(Lp, P, mode), (T, Lp)).reshape(-1)
+    real = np.zeros((T, Lp), dtype=bool)
+    real[:, :L] = True
+    real = real.reshape(-1)
+    mask = (cls[:, None] == cls[None, :]) & real[None, :]
+    N = T * Lp
+    out = np.zeros_like(qp)
+    for b in range(B):
+        for hd in range(heads):
+            Q = qp[b, :, :, hd, :].reshape(N, d)
+            K = kp[b, :, :, hd, :].reshape(N, d)
+            V = vp[b, :, :, hd, :].reshape(N, d)
+            S = (Q[real] @ K.T) / np.sqrt(d)
+            S = np.where(mask[real], S, -np.inf)
+            S = S - S.max(axis=1, keepdims=True)
+            E = np.exp(S)
+            O = np.zeros((N, d))
+            O[real] = (E / E.sum(axis=1, keepdims=True)) @ V
+            out[b, :, :, hd, :] = O.reshape(T, Lp, d)
+    return out[:, :, :L].reshape(B, T, H, W, heads, d)
+
+
+def attention_1d_torch(q, k, v, P: int, mode: int):
+    """attention_1d in torch fp64, differentiable. Returns (out, lse)."""
+    import torch
+    B, T, H, W, heads, d = q.shape
+    k2 = (P * P) ** 2
+    L = H * W
+    Lp = -(-L // k2) * k2
+    qp, kp, vp = (torch.nn.functional.pad(a.reshape(B, T, L, heads, d), (0, 0, 0, 0, 0, Lp - L))
+                  for a in (q, k, v))
+    cls = torch.from_numpy(np.broadcast_to(class_1d(Lp, P, mode), (T, Lp)).reshape(-1).copy())
+    real = torch.zeros((T, Lp), dtype=torch.bool)
+    real[:, :L] = True
+    real = real.reshape(-1)
+    mask = (cls[:, None] == cls[None, :]) & real[None, :]
+    N = T * Lp
+    outs, lses = [], []
+    for b in range(B):
+        ob, lb = [], []
+        for hd in range(heads):
+            Q = qp[b, :, :, hd, :].reshape(N, d)[real]
+            K = kp[b, :, :, hd, :].reshape(N, d)
+            V = vp[b, :, :, hd, :].reshape(N, d)
+            S = ((Q @ K.T) / (d ** 0.5)).masked_fill(~mask[real], float("-inf"))
+            lse = torch.logsumexp(S, dim=1)
+            ob.append(torch.exp(S - lse[:, None]) @ V)
+            lb.append(lse)
+        outs.append(torch.stack(ob, dim=1))
+        lses.append(torch.stack(lb, dim=1))
+    # real positions in (t, x) order are exactly the original tokens in (t, h, w) order
+    return (torch.stack(outs).reshape(B, T, H, W, heads, d),
+            torch.stack(lses).reshape(B, T, H, W, heads))

@@ -21,6 +21,9 @@
  * the bottom/right; rearranged layout (B*P^2, n, heads, d) with subsequence index
  * b*P^2 + ci*P + cj and tokens in (t, r, s) raster order; pad slots hold 0;
  * softmax scale 1/sqrt(d); no causal mask.
+ * Skiparse-1D, the variant the pages compare against (技术新颖性, 实验结果), follows the same
+ * three steps with the class rule on the flattened in-frame index (reading stated at
+ * oracle1d_padded_length below).
  */
 #include "skiparse_oracle.h"
 
@@ -77,113 +80,217 @@ long long oracle_subseq_len(int T, int H, int W, int P) {
     return (long long)T * (Hp / P) * (Wp / P);
 }
 
-/* Step 1 (方法步骤详情): rearrange into P^2 subsequences, pad, and record the mask. */
-int oracle_rearrange(const uint16_t* x, uint16_t* y, uint8_t* valid,
-                     int B, int T, int H, int W, int heads, int d, int P, int mode) {
+/* Skiparse-1D (技术新颖性 and 实验结果 on the summary page: the 1D skip pattern on the flattened
+ * sequence, which Skiparse-2D applies to each spatial axis instead). The pages give no formula;
+ * the reading taken here is the one-axis rule above on the flattened in-frame index
+ * x = h*W + w with ratio P^2, so that there are P^2 subsequences as in Skiparse-2D:
+ * token-wise class x mod P^2, group-wise class (x div P^2) mod P^2. Each frame's H*W
+ * positions are padded at the end to the next multiple of P^4 (the one-axis any-resolution
+ * rule with ratio P^2). */
+int oracle1d_padded_length(int L, int P) {
+    if (L < 1 || P < 1) return -1;
+    return oracle_padded_extent(L, P * P);
+}
+
+int oracle1d_index_map(int x, int P, int mode, int* cls, int* pos) {
+    if (P < 1) return -1;
+    return oracle_axis_map(x, P * P, mode, cls, pos);
+}
+
+long long oracle1d_subseq_len(int T, int H, int W, int P) {
+    if (T < 1 || H < 1 || W < 1 || P < 1) return -1;
+    const int Lp = oracle1d_padded_length(H * W, P);
+    return (long long)T * (Lp / (P * P));
+}
+
+/* ---- where every padded position goes ------------------------------------------
+ * Both patterns cut each frame's padded positions f in [0, F) into P^2 classes. The
+ * rearranged layout is (B*P^2, n, heads, d): subsequence b*P^2 + class, and inside it the
+ * tokens of the class in frame order t, then in the order of their position in the class. */
+typedef struct {
+    int dims;             /* 2: Skiparse-2D; 1: Skiparse-1D */
+    int B, T, H, W, heads, d, P, mode;
+    long long F;          /* padded positions per frame */
+    long long n;          /* subsequence length */
+    int Hp, Wp, R, S;     /* Skiparse-2D: padded extents and sub-grid extents Hp/P, Wp/P */
+} pattern;
+
+static int pattern_init(pattern* pt, int dims, int B, int T, int H, int W, int heads, int d,
+                        int P, int mode) {
     if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long row = (long long)heads * d;
-    for (int b = 0; b < B; ++b)
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < Hp; ++h)
-                for (int w = 0; w < Wp; ++w) {
-                    int ci, r, cj, s;
-                    oracle_axis_map(h, P, mode, &ci, &r);
-                    oracle_axis_map(w, P, mode, &cj, &s);
-                    const long long seq = (long long)b * P * P + ci * P + cj;
-                    const long long pos = ((long long)t * R + r) * S + s;
-                    const int real = (h < H) && (w < W);
-                    uint16_t* dst = y + (seq * n + pos) * row;
-                    if (real) {
-                        const long long tok = (((long long)b * T + t) * H + h) * W + w;
-                        for (long long e = 0; e < row; ++e) dst[e] = x[tok * row + e];
-                    } else {
-                        for (long long e = 0; e < row; ++e) dst[e] = 0;
-                    }
-                    if (valid) valid[seq * n + pos] = (uint8_t)real;
-                }
+    if (dims != 1 && dims != 2) return -1;
+    memset(pt, 0, sizeof *pt);
+    pt->dims = dims;
+    pt->B = B; pt->T = T; pt->H = H; pt->W = W; pt->heads = heads; pt->d = d;
+    pt->P = P; pt->mode = mode;
+    if (dims == 2) {
+        pt->Hp = oracle_padded_extent(H, P);
+        pt->Wp = oracle_padded_extent(W, P);
+        pt->R = pt->Hp / P;
+        pt->S = pt->Wp / P;
+        pt->F = (long long)pt->Hp * pt->Wp;
+        pt->n = oracle_subseq_len(T, H, W, P);
+    } else {
+        pt->F = oracle1d_padded_length(H * W, P);
+        pt->n = oracle1d_subseq_len(T, H, W, P);
+    }
     return 0;
 }
 
+/* Slot of padded position f of frame t of batch element b: subsequence *seq, position *pos.
+ * Returns 1 for a real token (then *tok is its index ((b*T + t)*H + h)*W + w in the original
+ * layout) and 0 for a pad slot. Skiparse-2D: f = h*Wp + w, class (ci, cj) from the two axis
+ * maps, subsequence b*P^2 + ci*P + cj, position (t, r, s) in raster order. Skiparse-1D:
+ * f = x = h*W + w, class c from the flattened-index map, subsequence b*P^2 + c, position
+ * t*(F/P^2) + the position inside the class. */
+static int pattern_slot(const pattern* pt, int b, int t, long long f, long long* seq,
+                        long long* pos, long long* tok) {
+    const long long q2 = (long long)pt->P * pt->P;
+    if (pt->dims == 2) {
+        const int h = (int)(f / pt->Wp), w = (int)(f % pt->Wp);
+        int ci, r, cj, s;
+        oracle_axis_map(h, pt->P, pt->mode, &ci, &r);
+        oracle_axis_map(w, pt->P, pt->mode, &cj, &s);
+        *seq = (long long)b * q2 + ci * pt->P + cj;
+        *pos = ((long long)t * pt->R + r) * pt->S + s;
+        if (h >= pt->H || w >= pt->W) return 0;
+        *tok = (((long long)b * pt->T + t) * pt->H + h) * pt->W + w;
+        return 1;
+    }
+    int c, s;
+    oracle1d_index_map((int)f, pt->P, pt->mode, &c, &s);
+    *seq = (long long)b * q2 + c;
+    *pos = (long long)t * (pt->F / q2) + s;
+    if (f >= (long long)pt->H * pt->W) return 0;
+    *tok = ((long long)b * pt->T + t) * ((long long)pt->H * pt->W) + f;
+    return 1;
+}
+
+/* Batch element, frame and padded position of token `tok` of the original layout. */
+static void pattern_locate(const pattern* pt, long long tok, int* b, int* t, long long* f) {
+    const long long hw = (long long)pt->H * pt->W;
+    const long long x = tok % hw;
+    *t = (int)((tok / hw) % pt->T);
+    *b = (int)(tok / (hw * pt->T));
+    *f = pt->dims == 2 ? (x / pt->W) * pt->Wp + x % pt->W : x;
+}
+
+/* Step 1 (方法步骤详情): rearrange into P^2 subsequences, pad, and record the mask. */
+static void rearrange_impl(const pattern* pt, const uint16_t* x, uint16_t* y, uint8_t* valid) {
+    const long long row = (long long)pt->heads * pt->d;
+    for (int b = 0; b < pt->B; ++b)
+        for (int t = 0; t < pt->T; ++t)
+            for (long long f = 0; f < pt->F; ++f) {
+                long long seq, pos, tok = 0;
+                const int real = pattern_slot(pt, b, t, f, &seq, &pos, &tok);
+                uint16_t* dst = y + (seq * pt->n + pos) * row;
+                for (long long e = 0; e < row; ++e) dst[e] = real ? x[tok * row + e] : 0;
+                if (valid) valid[seq * pt->n + pos] = (uint8_t)real;
+            }
+}
+
 /* Step 3 (方法步骤详情: rearrange back to the original layout), real tokens only. */
+static void unrearrange_impl(const pattern* pt, const void* y, void* x, int elem_bytes,
+                             long long row) {
+    for (int b = 0; b < pt->B; ++b)
+        for (int t = 0; t < pt->T; ++t)
+            for (long long f = 0; f < pt->F; ++f) {
+                long long seq, pos, tok = 0;
+                if (!pattern_slot(pt, b, t, f, &seq, &pos, &tok)) continue;
+                memcpy((char*)x + tok * row * elem_bytes,
+                       (const char*)y + (seq * pt->n + pos) * row * elem_bytes,
+                       (size_t)(row * elem_bytes));
+            }
+}
+
+/* Pattern switch between layers (核心方法: token-wise and group-wise alternate between layers;
+ * 方法步骤详情: under SSP a switch is a local rearrange plus one exchange). The local step: a
+ * tensor in the source mode's rearranged layout goes straight to the other mode's rearranged
+ * layout; every real token row moves from its source slot to its destination slot, pad slots
+ * of the result are 0. */
+static void switch_impl(const pattern* src, const pattern* dst, const uint16_t* ysrc,
+                        uint16_t* ydst) {
+    const long long row = (long long)src->heads * src->d;
+    for (int b = 0; b < dst->B; ++b)
+        for (int t = 0; t < dst->T; ++t)
+            for (long long f = 0; f < dst->F; ++f) {
+                long long dseq, dpos, sseq, spos, tok = 0;
+                const int real = pattern_slot(dst, b, t, f, &dseq, &dpos, &tok);
+                uint16_t* out = ydst + (dseq * dst->n + dpos) * row;
+                if (real) {
+                    pattern_slot(src, b, t, f, &sseq, &spos, &tok);
+                    for (long long e = 0; e < row; ++e) out[e] = ysrc[(sseq * src->n + spos) * row + e];
+                } else {
+                    for (long long e = 0; e < row; ++e) out[e] = 0;
+                }
+            }
+}
+
+int oracle_rearrange(const uint16_t* x, uint16_t* y, uint8_t* valid,
+                     int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    rearrange_impl(&pt, x, y, valid);
+    return 0;
+}
+
+int oracle1d_rearrange(const uint16_t* x, uint16_t* y, uint8_t* valid,
+                       int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    rearrange_impl(&pt, x, y, valid);
+    return 0;
+}
+
 int oracle_unrearrange(const uint16_t* y, uint16_t* x,
                        int B, int T, int H, int W, int heads, int d, int P, int mode) {
-    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long row = (long long)heads * d;
-    for (int b = 0; b < B; ++b)
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < H; ++h)
-                for (int w = 0; w < W; ++w) {
-                    int ci, r, cj, s;
-                    oracle_axis_map(h, P, mode, &ci, &r);
-                    oracle_axis_map(w, P, mode, &cj, &s);
-                    const long long seq = (long long)b * P * P + ci * P + cj;
-                    const long long pos = ((long long)t * R + r) * S + s;
-                    const long long tok = (((long long)b * T + t) * H + h) * W + w;
-                    for (long long e = 0; e < row; ++e) x[tok * row + e] = y[(seq * n + pos) * row + e];
-                }
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    unrearrange_impl(&pt, y, x, 2, (long long)heads * d);
+    return 0;
+}
+
+int oracle1d_unrearrange(const uint16_t* y, uint16_t* x,
+                         int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    unrearrange_impl(&pt, y, x, 2, (long long)heads * d);
     return 0;
 }
 
 int oracle_unrearrange_f64(const double* y, double* x,
                            int B, int T, int H, int W, int heads, int d, int P, int mode) {
-    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long row = (long long)heads * d;
-    for (int b = 0; b < B; ++b)
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < H; ++h)
-                for (int w = 0; w < W; ++w) {
-                    int ci, r, cj, s;
-                    oracle_axis_map(h, P, mode, &ci, &r);
-                    oracle_axis_map(w, P, mode, &cj, &s);
-                    const long long seq = (long long)b * P * P + ci * P + cj;
-                    const long long pos = ((long long)t * R + r) * S + s;
-                    const long long tok = (((long long)b * T + t) * H + h) * W + w;
-                    for (long long e = 0; e < row; ++e) x[tok * row + e] = y[(seq * n + pos) * row + e];
-                }
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    unrearrange_impl(&pt, y, x, 8, (long long)heads * d);
     return 0;
 }
 
-/* Pattern switch between layers (核心方法: token-wise and group-wise alternate between layers;
- * 方法步骤详情: under SSP a switch is a local rearrange plus one exchange). The local step: a
- * tensor in src_mode's rearranged layout goes straight to the other mode's rearranged layout;
- * every real token row moves from its src_mode slot to its dst_mode slot, pad slots of the
- * result are 0. */
+int oracle1d_unrearrange_f64(const double* y, double* x,
+                             int B, int T, int H, int W, int heads, int d, int P, int mode) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    unrearrange_impl(&pt, y, x, 8, (long long)heads * d);
+    return 0;
+}
+
+static int switch_dims(int dims, const uint16_t* ysrc, uint16_t* ydst, int B, int T, int H,
+                       int W, int heads, int d, int P, int src_mode) {
+    pattern src, dst;
+    if (pattern_init(&src, dims, B, T, H, W, heads, d, P, src_mode)) return -1;
+    if (pattern_init(&dst, dims, B, T, H, W, heads, d, P, 1 - src_mode)) return -1;
+    switch_impl(&src, &dst, ysrc, ydst);
+    return 0;
+}
+
 int oracle_switch_mode(const uint16_t* ysrc, uint16_t* ydst,
                        int B, int T, int H, int W, int heads, int d, int P, int src_mode) {
-    if (check_shape(B, T, H, W, heads, d, P, src_mode)) return -1;
-    const int dst_mode = 1 - src_mode;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long row = (long long)heads * d;
-    for (int b = 0; b < B; ++b)
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < Hp; ++h)
-                for (int w = 0; w < Wp; ++w) {
-                    int ci, r, cj, s;
-                    oracle_axis_map(h, P, dst_mode, &ci, &r);
-                    oracle_axis_map(w, P, dst_mode, &cj, &s);
-                    const long long dslot = ((long long)b * P * P + ci * P + cj) * n + ((long long)t * R + r) * S + s;
-                    uint16_t* dst = ydst + dslot * row;
-                    if (h < H && w < W) {
-                        oracle_axis_map(h, P, src_mode, &ci, &r);
-                        oracle_axis_map(w, P, src_mode, &cj, &s);
-                        const long long sslot = ((long long)b * P * P + ci * P + cj) * n + ((long long)t * R + r) * S + s;
-                        for (long long e = 0; e < row; ++e) dst[e] = ysrc[sslot * row + e];
-                    } else {
-                        for (long long e = 0; e < row; ++e) dst[e] = 0;
-                    }
-                }
-    return 0;
+    return switch_dims(2, ysrc, ydst, B, T, H, W, heads, d, P, src_mode);
+}
+
+int oracle1d_switch_mode(const uint16_t* ysrc, uint16_t* ydst,
+                         int B, int T, int H, int W, int heads, int d, int P, int src_mode) {
+    return switch_dims(1, ysrc, ydst, B, T, H, W, heads, d, P, src_mode);
 }
 
 /* Step 2: dense softmax attention of one query row over the real keys of its own
@@ -295,41 +402,52 @@ static void free_rearranged(rearranged* r) {
     free(r->yq); free(r->yk); free(r->yv); free(r->valid);
 }
 
-static int rearrange_all(const uint16_t* q, const uint16_t* k, const uint16_t* v, rearranged* r,
-                         int B, int T, int H, int W, int heads, int d, int P, int mode,
-                         long long* n_out) {
-    const long long n = oracle_subseq_len(T, H, W, P);
-    const long long nseq = (long long)B * P * P;
-    const size_t elems = (size_t)(nseq * n * heads * d);
+static int rearrange_all(const pattern* pt, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, rearranged* r) {
+    const long long nseq = (long long)pt->B * pt->P * pt->P;
+    const size_t elems = (size_t)(nseq * pt->n * pt->heads * pt->d);
     memset(r, 0, sizeof *r);
     r->yq = (uint16_t*)malloc(elems * 2);
     r->yk = (uint16_t*)malloc(elems * 2);
     r->yv = (uint16_t*)malloc(elems * 2);
-    r->valid = (uint8_t*)malloc((size_t)(nseq * n));
+    r->valid = (uint8_t*)malloc((size_t)(nseq * pt->n));
     if (!r->yq || !r->yk || !r->yv || !r->valid) { free_rearranged(r); return -2; }
-    oracle_rearrange(q, r->yq, r->valid, B, T, H, W, heads, d, P, mode);
-    oracle_rearrange(k, r->yk, NULL, B, T, H, W, heads, d, P, mode);
-    oracle_rearrange(v, r->yv, NULL, B, T, H, W, heads, d, P, mode);
-    *n_out = n;
+    rearrange_impl(pt, q, r->yq, r->valid);
+    rearrange_impl(pt, k, r->yk, NULL);
+    rearrange_impl(pt, v, r->yv, NULL);
     return 0;
+}
+
+static int attn_fwd_impl(const pattern* pt, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, double* out, int nthreads) {
+    rearranged r;
+    int rc = rearrange_all(pt, q, k, v, &r);
+    if (rc) return rc;
+    const long long nseq = (long long)pt->B * pt->P * pt->P;
+    double* yo = (double*)calloc((size_t)(nseq * pt->n * pt->heads * pt->d), sizeof(double));
+    if (!yo) { free_rearranged(&r); return -2; }
+    rc = oracle_masked_attention(r.yq, r.yk, r.yv, r.valid, yo, nseq, pt->n, pt->heads, pt->d,
+                                 nthreads);
+    if (!rc) unrearrange_impl(pt, yo, out, 8, (long long)pt->heads * pt->d);
+    free(yo);
+    free_rearranged(&r);
+    return rc;
 }
 
 int oracle_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, double* out,
                     int B, int T, int H, int W, int heads, int d, int P, int mode,
                     int nthreads) {
-    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
-    rearranged r;
-    long long n = 0;
-    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
-    if (rc) return rc;
-    const long long nseq = (long long)B * P * P;
-    double* yo = (double*)calloc((size_t)(nseq * n * heads * d), sizeof(double));
-    if (!yo) { free_rearranged(&r); return -2; }
-    rc = oracle_masked_attention(r.yq, r.yk, r.yv, r.valid, yo, nseq, n, heads, d, nthreads);
-    if (!rc) rc = oracle_unrearrange_f64(yo, out, B, T, H, W, heads, d, P, mode);
-    free(yo);
-    free_rearranged(&r);
-    return rc;
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_fwd_impl(&pt, q, k, v, out, nthreads);
+}
+
+int oracle1d_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, double* out,
+                      int B, int T, int H, int W, int heads, int d, int P, int mode,
+                      int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_fwd_impl(&pt, q, k, v, out, nthreads);
 }
 
 /* The forward pass for selected output rows. The pages' three steps restricted to what
@@ -367,39 +485,61 @@ static int cmp_ll(const void* a, const void* b) {
     return x < y ? -1 : x > y;
 }
 
-int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                         const long long* rows, long long nrows, double* out_rows,
-                         int B, int T, int H, int W, int heads, int d, int P, int mode,
-                         int nthreads) {
-    if (check_shape(B, T, H, W, heads, d, P, mode) || nrows < 0) return -1;
-    const long long ntok = (long long)B * T * H * W;
-    for (long long i = 0; i < nrows; ++i)
-        if (rows[i] < 0 || rows[i] >= ntok * heads) return -1;
-    if (nrows == 0) return 0;
-    if (nthreads < 1) nthreads = 1;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long q2 = (long long)P * P;
-    /* key = ((seq*heads + head) * n + pos), packed with the request index for sorting */
+/* Sort key of each requested row: ((subsequence*heads + head) * n + position), with the
+ * request's index beside it, so that the requests of one (subsequence, head) are adjacent. */
+static long long* request_keys(const pattern* pt, const long long* rows, long long nrows) {
     long long* key = (long long*)malloc(sizeof(long long) * (size_t)nrows * 2);
-    if (!key) return -2;
+    if (!key) return NULL;
     for (long long i = 0; i < nrows; ++i) {
-        const int head = (int)(rows[i] % heads);
-        long long tok = rows[i] / heads;
-        const int w = (int)(tok % W); tok /= W;
-        const int h = (int)(tok % H); tok /= H;
-        const int t = (int)(tok % T);
-        const int b = (int)(tok / T);
-        int ci, rr, cj, ss;
-        oracle_axis_map(h, P, mode, &ci, &rr);
-        oracle_axis_map(w, P, mode, &cj, &ss);
-        const long long seq = (long long)b * q2 + ci * P + cj;
-        const long long pos = ((long long)t * R + rr) * S + ss;
-        key[2 * i] = (seq * heads + head) * n + pos;
+        const int head = (int)(rows[i] % pt->heads);
+        int b, t;
+        long long f, seq, pos, tok;
+        pattern_locate(pt, rows[i] / pt->heads, &b, &t, &f);
+        pattern_slot(pt, b, t, f, &seq, &pos, &tok);
+        key[2 * i] = (seq * pt->heads + head) * pt->n + pos;
         key[2 * i + 1] = i;
     }
     qsort(key, (size_t)nrows, 2 * sizeof(long long), cmp_ll);
+    return key;
+}
+
+/* Step 1 for one subsequence and one head: the same slot rule as rearrange_impl, keeping only
+ * the slots of subsequence `seq`. Any of the destination buffers may be NULL. */
+static void gather_subseq(const pattern* pt, long long seq, int head, const uint16_t* const* src,
+                          uint16_t* const* dst, int nbuf, uint8_t* valid) {
+    const long long q2 = (long long)pt->P * pt->P;
+    const int b = (int)(seq / q2);
+    const int d = pt->d;
+    for (int t = 0; t < pt->T; ++t)
+        for (long long f = 0; f < pt->F; ++f) {
+            long long s, p, tok = 0;
+            const int real = pattern_slot(pt, b, t, f, &s, &p, &tok);
+            if (s != seq) continue;
+            valid[p] = (uint8_t)real;
+            const long long srow = tok * pt->heads + head;
+            for (int i = 0; i < nbuf; ++i)
+                for (int e = 0; e < d; ++e) dst[i][p * d + e] = real ? src[i][srow * d + e] : 0;
+        }
+}
+
+static int check_rows(const pattern* pt, const long long* rows, long long nrows) {
+    const long long ntok = (long long)pt->B * pt->T * pt->H * pt->W;
+    if (nrows < 0) return -1;
+    for (long long i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= ntok * pt->heads) return -1;
+    return 0;
+}
+
+static int attn_fwd_rows_impl(const pattern* pt, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const long long* rows, long long nrows,
+                              double* out_rows, int nthreads) {
+    if (check_rows(pt, rows, nrows)) return -1;
+    if (nrows == 0) return 0;
+    if (nthreads < 1) nthreads = 1;
+    const long long n = pt->n;
+    const int heads = pt->heads, d = pt->d;
+    long long* key = request_keys(pt, rows, nrows);
+    if (!key) return -2;
     uint16_t* sq = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
     uint16_t* sk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
     uint16_t* sv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
@@ -418,28 +558,9 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
             slot[g1 - g0] = key[2 * g1 + 1];
             ++g1;
         }
-        const long long seq = group / heads;
-        const int head = (int)(group % heads);
-        const int b = (int)(seq / q2);
-        const int c = (int)(seq % q2);
-        /* step 1 for this subsequence and head: same loops as oracle_rearrange */
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < Hp; ++h)
-                for (int w = 0; w < Wp; ++w) {
-                    int ci, rr, cj, ss;
-                    oracle_axis_map(h, P, mode, &ci, &rr);
-                    oracle_axis_map(w, P, mode, &cj, &ss);
-                    if (ci * P + cj != c) continue;
-                    const long long p = ((long long)t * R + rr) * S + ss;
-                    const int real = (h < H) && (w < W);
-                    valid[p] = (uint8_t)real;
-                    const long long src = ((((long long)b * T + t) * H + h) * W + w) * heads + head;
-                    for (int e = 0; e < d; ++e) {
-                        sq[p * d + e] = real ? q[src * d + e] : 0;
-                        sk[p * d + e] = real ? k[src * d + e] : 0;
-                        sv[p * d + e] = real ? v[src * d + e] : 0;
-                    }
-                }
+        const uint16_t* src[3] = {q, k, v};
+        uint16_t* dst[3] = {sq, sk, sv};
+        gather_subseq(pt, group / heads, (int)(group % heads), src, dst, 3, valid);
         /* step 2 for the requested queries, step 3 by writing to their slots */
         int started = 0;
         for (int t = 0; t < nthreads; ++t) {
@@ -459,6 +580,24 @@ int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
     }
     free(key); free(sq); free(sk); free(sv); free(valid); free(pos); free(slot); free(th); free(jobs);
     return rc;
+}
+
+int oracle_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         const long long* rows, long long nrows, double* out_rows,
+                         int B, int T, int H, int W, int heads, int d, int P, int mode,
+                         int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_fwd_rows_impl(&pt, q, k, v, rows, nrows, out_rows, nthreads);
+}
+
+int oracle1d_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const long long* rows, long long nrows, double* out_rows,
+                           int B, int T, int H, int W, int heads, int d, int P, int mode,
+                           int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_fwd_rows_impl(&pt, q, k, v, rows, nrows, out_rows, nthreads);
 }
 
 
@@ -544,16 +683,16 @@ static void* bwd_worker(void* arg) {
     return NULL;
 }
 
-int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
-                    double* dq, double* dk, double* dv, double* lse,
-                    int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads) {
-    if (check_shape(B, T, H, W, heads, d, P, mode)) return -1;
+static int attn_bwd_impl(const pattern* pt, const uint16_t* q, const uint16_t* k,
+                         const uint16_t* v, const uint16_t* dout, double* dq, double* dk,
+                         double* dv, double* lse, int nthreads) {
     if (nthreads < 1) nthreads = 1;
     rearranged r;
-    long long n = 0;
-    int rc = rearrange_all(q, k, v, &r, B, T, H, W, heads, d, P, mode, &n);
+    int rc = rearrange_all(pt, q, k, v, &r);
     if (rc) return rc;
-    const long long nseq = (long long)B * P * P;
+    const long long n = pt->n;
+    const int heads = pt->heads, d = pt->d;
+    const long long nseq = (long long)pt->B * pt->P * pt->P;
     const size_t elems = (size_t)(nseq * n * heads * d);
     uint16_t* ydo = (uint16_t*)malloc(elems * 2);
     double* ydq = (double*)calloc(elems, sizeof(double));
@@ -564,7 +703,7 @@ int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, con
     bwd_job* jobs = (bwd_job*)malloc(sizeof(bwd_job) * (size_t)nthreads);
     if (!ydo || !ydq || !ydk || !ydv || (lse && !ylse) || !th || !jobs) rc = -2;
     if (!rc) {
-        oracle_rearrange(dout, ydo, NULL, B, T, H, W, heads, d, P, mode);
+        rearrange_impl(pt, dout, ydo, NULL);
         int started = 0;
         for (int t = 0; t < nthreads; ++t) {
             bwd_job* jb = &jobs[t];
@@ -582,14 +721,31 @@ int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, con
         }
     }
     if (!rc) {
-        oracle_unrearrange_f64(ydq, dq, B, T, H, W, heads, d, P, mode);
-        oracle_unrearrange_f64(ydk, dk, B, T, H, W, heads, d, P, mode);
-        oracle_unrearrange_f64(ydv, dv, B, T, H, W, heads, d, P, mode);
-        if (lse) oracle_unrearrange_f64(ylse, lse, B, T, H, W, heads, 1, P, mode);
+        const long long row = (long long)heads * d;
+        unrearrange_impl(pt, ydq, dq, 8, row);
+        unrearrange_impl(pt, ydk, dk, 8, row);
+        unrearrange_impl(pt, ydv, dv, 8, row);
+        if (lse) unrearrange_impl(pt, ylse, lse, 8, heads);
     }
     free(ydo); free(ydq); free(ydk); free(ydv); free(ylse); free(th); free(jobs);
     free_rearranged(&r);
     return rc;
+}
+
+int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                    double* dq, double* dk, double* dv, double* lse,
+                    int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_bwd_impl(&pt, q, k, v, dout, dq, dk, dv, lse, nthreads);
+}
+
+int oracle1d_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                      double* dq, double* dk, double* dv, double* lse,
+                      int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_bwd_impl(&pt, q, k, v, dout, dq, dk, dv, lse, nthreads);
 }
 
 /* Gradients for selected rows (token*heads + head of the original layout): dq of the token as
@@ -694,37 +850,17 @@ static int run_bwdrows(bwdrows_job proto, int nthreads, int phase) {
     return rc;
 }
 
-int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
-                         const long long* rows, long long nrows, double* dq_rows, double* dk_rows,
-                         double* dv_rows, int B, int T, int H, int W, int heads, int d, int P,
-                         int mode, int nthreads) {
-    if (check_shape(B, T, H, W, heads, d, P, mode) || nrows < 0) return -1;
-    const long long ntok = (long long)B * T * H * W;
-    for (long long i = 0; i < nrows; ++i)
-        if (rows[i] < 0 || rows[i] >= ntok * heads) return -1;
+static int attn_bwd_rows_impl(const pattern* pt, const uint16_t* q, const uint16_t* k,
+                              const uint16_t* v, const uint16_t* dout, const long long* rows,
+                              long long nrows, double* dq_rows, double* dk_rows, double* dv_rows,
+                              int nthreads) {
+    if (check_rows(pt, rows, nrows)) return -1;
     if (nrows == 0) return 0;
     if (nthreads < 1) nthreads = 1;
-    const int Hp = oracle_padded_extent(H, P), Wp = oracle_padded_extent(W, P);
-    const int R = Hp / P, S = Wp / P;
-    const long long n = (long long)T * R * S;
-    const long long q2 = (long long)P * P;
-    long long* key = (long long*)malloc(sizeof(long long) * (size_t)nrows * 2);
+    const long long n = pt->n;
+    const int heads = pt->heads, d = pt->d;
+    long long* key = request_keys(pt, rows, nrows);
     if (!key) return -2;
-    for (long long i = 0; i < nrows; ++i) {
-        const int head = (int)(rows[i] % heads);
-        long long tok = rows[i] / heads;
-        const int w = (int)(tok % W); tok /= W;
-        const int h = (int)(tok % H); tok /= H;
-        const int t = (int)(tok % T);
-        const int b = (int)(tok / T);
-        int ci, rr, cj, ss;
-        oracle_axis_map(h, P, mode, &ci, &rr);
-        oracle_axis_map(w, P, mode, &cj, &ss);
-        const long long seq = (long long)b * q2 + ci * P + cj;
-        key[2 * i] = (seq * heads + head) * n + ((long long)t * R + rr) * S + ss;
-        key[2 * i + 1] = i;
-    }
-    qsort(key, (size_t)nrows, 2 * sizeof(long long), cmp_ll);
     uint16_t* sq = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
     uint16_t* sk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
     uint16_t* sv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * d));
@@ -744,28 +880,9 @@ int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
             slot[g1 - g0] = key[2 * g1 + 1];
             ++g1;
         }
-        const long long seq = group / heads;
-        const int head = (int)(group % heads);
-        const int b = (int)(seq / q2);
-        const int c = (int)(seq % q2);
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < Hp; ++h)
-                for (int w = 0; w < Wp; ++w) {
-                    int ci, rr, cj, ss;
-                    oracle_axis_map(h, P, mode, &ci, &rr);
-                    oracle_axis_map(w, P, mode, &cj, &ss);
-                    if (ci * P + cj != c) continue;
-                    const long long pp = ((long long)t * R + rr) * S + ss;
-                    const int real = (h < H) && (w < W);
-                    valid[pp] = (uint8_t)real;
-                    const long long src = ((((long long)b * T + t) * H + h) * W + w) * heads + head;
-                    for (int e = 0; e < d; ++e) {
-                        sq[pp * d + e] = real ? q[src * d + e] : 0;
-                        sk[pp * d + e] = real ? k[src * d + e] : 0;
-                        sv[pp * d + e] = real ? v[src * d + e] : 0;
-                        sdo[pp * d + e] = real ? dout[src * d + e] : 0;
-                    }
-                }
+        const uint16_t* src[4] = {q, k, v, dout};
+        uint16_t* dst[4] = {sq, sk, sv, sdo};
+        gather_subseq(pt, group / heads, (int)(group % heads), src, dst, 4, valid);
         bwdrows_job jb;
         memset(&jb, 0, sizeof jb);
         jb.sq = sq; jb.sk = sk; jb.sv = sv; jb.sdo = sdo; jb.valid = valid;
@@ -778,4 +895,22 @@ int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
     }
     free(key); free(sq); free(sk); free(sv); free(sdo); free(valid); free(L); free(Dl); free(pos); free(slot);
     return rc;
+}
+
+int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                         const long long* rows, long long nrows, double* dq_rows, double* dk_rows,
+                         double* dv_rows, int B, int T, int H, int W, int heads, int d, int P,
+                         int mode, int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 2, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_bwd_rows_impl(&pt, q, k, v, dout, rows, nrows, dq_rows, dk_rows, dv_rows, nthreads);
+}
+
+int oracle1d_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* dout, const long long* rows, long long nrows,
+                           double* dq_rows, double* dk_rows, double* dv_rows, int B, int T, int H,
+                           int W, int heads, int d, int P, int mode, int nthreads) {
+    pattern pt;
+    if (pattern_init(&pt, 1, B, T, H, W, heads, d, P, mode)) return -1;
+    return attn_bwd_rows_impl(&pt, q, k, v, dout, rows, nrows, dq_rows, dk_rows, dv_rows, nthreads);
 }

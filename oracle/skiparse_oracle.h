@@ -1,7 +1,7 @@
 /*
  * skiparse_oracle.h -- TEST INFRASTRUCTURE ONLY.
  *
- * Plain, slow, fp64 CPU oracle for Skiparse-2D sparse attention (OSP-Next). Only the
+ * Plain, slow, fp64 CPU oracle for Skiparse-2D (and Skiparse-1D) sparse attention (OSP-Next). Only the
  * test suite, the smoke check and the benchmark's CPU-baseline leg may call it. It
  * shares no code, header or constant with the CUDA library in fixed_pattern_sparse_b200/.
  *
@@ -83,6 +83,39 @@ int oracle_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
                          const long long* rows, long long nrows, double* dq_rows, double* dk_rows,
                          double* dv_rows, int B, int T, int H, int W, int heads, int d, int P,
                          int mode, int nthreads);
+
+/* ---- Skiparse-1D (the 1D skip pattern on the flattened sequence; summary page sections
+ * 技术新颖性 and 实验结果 compare it with Skiparse-2D but give no formula). Reading: the one-axis
+ * rule above applied to the in-frame index x = h*W + w with ratio P^2 -- token-wise class
+ * x mod P^2, group-wise class (x div P^2) mod P^2 -- and each frame's H*W positions padded at
+ * the end to a multiple of P^4. The rearranged layout is (B*P*P, n, heads, d) with
+ * n = T * Lp / P^2, subsequence b*P^2 + class, tokens in (t, position-in-class) order.
+ * Arguments and return values as for the Skiparse-2D functions of the same name. */
+int oracle1d_padded_length(int L, int P);
+int oracle1d_index_map(int x, int P, int mode, int* cls, int* pos);
+long long oracle1d_subseq_len(int T, int H, int W, int P);
+int oracle1d_rearrange(const uint16_t* x, uint16_t* y, uint8_t* valid,
+                       int B, int T, int H, int W, int heads, int d, int P, int mode);
+int oracle1d_unrearrange(const uint16_t* y, uint16_t* x,
+                         int B, int T, int H, int W, int heads, int d, int P, int mode);
+int oracle1d_unrearrange_f64(const double* y, double* x,
+                             int B, int T, int H, int W, int heads, int d, int P, int mode);
+int oracle1d_switch_mode(const uint16_t* ysrc, uint16_t* ydst,
+                         int B, int T, int H, int W, int heads, int d, int P, int src_mode);
+int oracle1d_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, double* out,
+                      int B, int T, int H, int W, int heads, int d, int P, int mode,
+                      int nthreads);
+int oracle1d_attn_fwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const long long* rows, long long nrows, double* out_rows,
+                           int B, int T, int H, int W, int heads, int d, int P, int mode,
+                           int nthreads);
+int oracle1d_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                      double* dq, double* dk, double* dv, double* lse,
+                      int B, int T, int H, int W, int heads, int d, int P, int mode, int nthreads);
+int oracle1d_attn_bwd_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const uint16_t* dout, const long long* rows, long long nrows,
+                           double* dq_rows, double* dk_rows, double* dv_rows, int B, int T, int H,
+                           int W, int heads, int d, int P, int mode, int nthreads);
 
 #ifdef __cplusplus
 }
