@@ -340,6 +340,41 @@ def run_ours(args):
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the dense comparison")
 
+    # Skiparse-1D (the flattened-sequence variant) at the same shape on the same kernels: the
+    # 1D-vs-2D comparison, by the same padded FLOP formula with N = T * Lp
+    one_d = None
+    if not args.no_1d and w.P > 1:
+        fl1 = fps.attn_flops(q.shape, w.P, dims=1)
+        for i in range(3):
+            fps.skiparse1d_attn_fwd(qd, kd, vd, w.P, modes[i % len(modes)], out=out)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.one_d_steps):
+            fps.skiparse1d_attn_fwd(qd, kd, vd, w.P, modes[i % len(modes)], out=out)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms1 = e0.elapsed_time(e1) / args.one_d_steps
+        yshape1 = fps.rearranged_shape(q.shape, w.P, dims=1)
+        y1 = torch.empty(yshape1, dtype=torch.bfloat16, device=dev)
+        for i in range(3):
+            fps.skiparse1d_rearrange(qd, w.P, modes[i % len(modes)], out=y1)
+        e0.record(stream)
+        for i in range(args.rearrange_steps):
+            fps.skiparse1d_rearrange(qd, w.P, modes[i % len(modes)], out=y1)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        rms1 = e0.elapsed_time(e1) / args.rearrange_steps
+        rbytes1 = (qd.numel() + y1.numel()) * 2
+        del y1
+        if fps.get_device_status() != 0:
+            raise SystemExit("device status error in the Skiparse-1D timing")
+        one_d = {"ms_per_layer": round(ms1, 3), "tflops": round(fl1 / (ms1 / 1e3) / 1e12, 1),
+                 "frac_of_bf16_peak": round(fl1 / (ms1 / 1e3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+                 "padded_tokens_per_frame": fps.padded_length_1d(w.H * w.W, w.P),
+                 "vs_2d_ms": round(ms1 / statistics.mean(per_launch), 3),
+                 "rearrange_gbs": round(rbytes1 / (rms1 / 1e3) / 1e9, 1),
+                 "modes": "alternating " + " / ".join(MODE_NAME[m] for m in modes)}
+
     # backward pass (fine-tuning): 3 launches per call, FLOPs counted as 2.5x the forward's
     # (dV, dP, dQ, dK and the recomputed S: the standard accounting of attention backward)
     bwd = None
@@ -434,6 +469,7 @@ def run_ours(args):
             "ms_per_layer": {k_: round(v_, 3) for k_, v_ in by_mode.items()},
             "tflops_real_pairs": real,
             "dense_p1": dense,
+            "skiparse1d": one_d,
             "rearrange_kernels": rearr,
             "backward": bwd,
             "kernel_hash": kernel_hash(),
@@ -580,6 +616,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rearrange", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-1d", action="store_true", help="skip the Skiparse-1D comparison")
+    ap.add_argument("--one-d-steps", type=int, default=4)
     ap.add_argument("--backward-steps", type=int, default=4)
     ap.add_argument("--rearrange-steps", type=int, default=10)
     ap.add_argument("--stack", action="store_true",

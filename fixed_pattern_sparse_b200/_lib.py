@@ -33,6 +33,16 @@ SIGNATURES = {
     "skiparse_set_wait_limit_ns": (_ULL, [_ULL]),
     "skiparse_debug_inject_fault": (_I, [_I]),
     "skiparse_debug_exp2": (_I, [_VP, _VP, _LL, _I, _VP]),
+    "skiparse1d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse1d_attn_fwd_lse": (_I, [_VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse1d_attn_bwd": (_I, [_VP] * 10 + [_I] * 8 + [_VP]),
+    "skiparse1d_rearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse1d_unrearrange": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse1d_switch_mode": (_I, [_VP, _VP] + [_I] * 8 + [_VP]),
+    "skiparse1d_padded_length": (_LL, [_LL, _I]),
+    "skiparse1d_subseq_len": (_LL, [_I] * 4),
+    "skiparse1d_class_len": (_LL, [_I] * 6),
+    "skiparse1d_rearranged_numel": (_LL, [_I] * 7),
 }
 
 STATUS = {0: "SKIPARSE_OK", 1: "SKIPARSE_ERR_INVALID_ARG", 2: "SKIPARSE_ERR_UNSUPPORTED",

@@ -83,14 +83,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
     const int tile = blockIdx.x;
     const int head = blockIdx.y;
     const int seq = blockIdx.z;
-    const int q2 = p.P * p.P;
-    const int b = seq / q2, c = seq % q2, ci = c / p.P, cj = c % p.P;
+    const int q2 = p.Ph * p.Pw;
+    const int b = seq / q2, c = seq % q2, ci = c / p.Pw, cj = c % p.Pw;
     const int Rc = p.Rc[ci], Sc = p.Sc[cj];
     const int n_c = p.T * Rc * Sc;
     const int first = tile * kTileRows;
     if (first >= n_c) return;  // uniform over the CTA, before any shared state
     const int nstream = (n_c + kTileRows - 1) / kTileRows;
-    const RowMap rows{p.T, p.H, p.W, p.heads, p.P, p.mode, ci, cj, Rc, Sc, b, head};
+    const RowMap rows{p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head};
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = ptx::smem_u32(smem_raw);
@@ -407,12 +407,12 @@ int launch_bwd_d(const BwdParams& p, const Geometry& g, cudaStream_t stream) {
         attr_done_dev[dev] = 1;
     }
     int n_max = 0;
-    for (int ci = 0; ci < g.P; ++ci)
-        for (int cj = 0; cj < g.P; ++cj) {
+    for (int ci = 0; ci < g.Ph; ++ci)
+        for (int cj = 0; cj < g.Pw; ++cj) {
             const int n_c = g.T * g.Rc[ci] * g.Sc[cj];
             n_max = n_c > n_max ? n_c : n_max;
         }
-    dim3 grid((n_max + kTileRows - 1) / kTileRows, g.heads, g.B * g.P * g.P);
+    dim3 grid((n_max + kTileRows - 1) / kTileRows, g.heads, g.B * g.Ph * g.Pw);
     skiparse_attn_bwd_kernel<D, KV><<<grid, kBwdThreads, C::SMEM_BYTES, stream>>>(p);
     return static_cast<int>(cudaGetLastError());
 }

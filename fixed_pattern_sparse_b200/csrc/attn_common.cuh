@@ -33,15 +33,15 @@ struct TileGeom {
 
 // Global row (token*heads + head) of the class-local real token i of (b, ci, cj).
 struct RowMap {
-    int T, H, W, heads, P, mode;
+    int T, H, W, heads, Ph, Pw, mode;
     int ci, cj, Rc, Sc, b, head;
     __device__ __forceinline__ int operator()(int i) const {
         const int s = i % Sc;
         const int tr = i / Sc;
         const int r = tr % Rc;
         const int t = tr / Rc;
-        const int h = axis_coord(r, ci, P, mode);
-        const int w = axis_coord(s, cj, P, mode);
+        const int h = axis_coord(r, ci, Ph, mode);
+        const int w = axis_coord(s, cj, Pw, mode);
         return (((b * T + t) * H + h) * W + w) * heads + head;
     }
 };

@@ -148,14 +148,14 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
     const int pair = blockIdx.x;
     const int head = blockIdx.y;
     const int seq = blockIdx.z;
-    const int q2 = p.P * p.P;
-    const int b = seq / q2, c = seq % q2, ci = c / p.P, cj = c % p.P;
+    const int q2 = p.Ph * p.Pw;
+    const int b = seq / q2, c = seq % q2, ci = c / p.Pw, cj = c % p.Pw;
     const int Rc = p.Rc[ci], Sc = p.Sc[cj];
     const int n_c = p.T * Rc * Sc;
     const int q_first = pair * 2 * kBM;
     if (q_first >= n_c) return;  // uniform over the CTA, before any shared state
     const int nkv = (n_c + kBN - 1) / kBN;
-    const RowMap rows{p.T, p.H, p.W, p.heads, p.P, p.mode, ci, cj, Rc, Sc, b, head};
+    const RowMap rows{p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head};
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = ptx::smem_u32(smem_raw);
@@ -528,12 +528,12 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
         attr_done_dev[dev] = 1;
     }
     int n_max = 0;
-    for (int ci = 0; ci < g.P; ++ci)
-        for (int cj = 0; cj < g.P; ++cj) {
+    for (int ci = 0; ci < g.Ph; ++ci)
+        for (int cj = 0; cj < g.Pw; ++cj) {
             const int n_c = g.T * g.Rc[ci] * g.Sc[cj];
             n_max = n_c > n_max ? n_c : n_max;
         }
-    dim3 grid((n_max + 2 * kBM - 1) / (2 * kBM), g.heads, g.B * g.P * g.P);
+    dim3 grid((n_max + 2 * kBM - 1) / (2 * kBM), g.heads, g.B * g.Ph * g.Pw);
     skiparse_attn_fwd_kernel<D><<<grid, kThreads, C::SMEM_BYTES, stream>>>(p);
     return static_cast<int>(cudaGetLastError());
 }

@@ -9,7 +9,8 @@
 // mode's rearranged layout straight to the other's. All three are permutations of whole token
 // rows of heads*d bf16 values (contiguous in every layout), so the kernels are pure HBM copies:
 // one warp moves one row with 16-byte loads and stores, several chunks in flight per lane; pad
-// rows of a rearranged result are written as zero.
+// rows of a rearranged result are written as zero. Skiparse-1D uses the same kernels on a
+// (1, H*W) frame with (1, P^2) classes.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -45,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
     const int lane = threadIdx.x & 31;
     const long long warp0 = (static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const long long nwarps = (static_cast<long long>(gridDim.x) * kThreads) >> 5;
-    const int q2 = p.P * p.P;
+    const int q2 = p.Ph * p.Pw;
     const uint4* src = static_cast<const uint4*>(p.src);
     uint4* dst = static_cast<uint4*>(p.dst);
     for (long long row = warp0; row < p.nrows; row += nwarps) {
@@ -61,18 +62,18 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
             const long long tr = pos / p.S;
             const int r = static_cast<int>(tr % p.R);
             const int t = static_cast<int>(tr / p.R);
-            const int h = axis_coord(r, c / p.P, p.P, out_mode);
-            const int w = axis_coord(s, c % p.P, p.P, out_mode);
+            const int h = axis_coord(r, c / p.Pw, p.Ph, out_mode);
+            const int w = axis_coord(s, c % p.Pw, p.Pw, out_mode);
             real = h < p.H && w < p.W;
             if (kKind == 0) {
                 src_row = ((static_cast<long long>(b) * p.T + t) * p.H + h) * p.W + w;
             } else {
                 int ci = 0, r2 = 0, cj = 0, s2 = 0;
                 if (real) {
-                    axis_class(h, p.P, p.mode, ci, r2);
-                    axis_class(w, p.P, p.mode, cj, s2);
+                    axis_class(h, p.Ph, p.mode, ci, r2);
+                    axis_class(w, p.Pw, p.mode, cj, s2);
                 }
-                const long long sseq = static_cast<long long>(b) * q2 + ci * p.P + cj;
+                const long long sseq = static_cast<long long>(b) * q2 + ci * p.Pw + cj;
                 src_row = sseq * p.n + (static_cast<long long>(t) * p.R + r2) * p.S + s2;
             }
         } else {
@@ -84,9 +85,9 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
             const int t = static_cast<int>(tok % p.T);
             const int b = static_cast<int>(tok / p.T);
             int ci, r, cj, s;
-            axis_class(h, p.P, p.mode, ci, r);
-            axis_class(w, p.P, p.mode, cj, s);
-            const long long seq = static_cast<long long>(b) * q2 + ci * p.P + cj;
+            axis_class(h, p.Ph, p.mode, ci, r);
+            axis_class(w, p.Pw, p.mode, cj, s);
+            const long long seq = static_cast<long long>(b) * q2 + ci * p.Pw + cj;
             src_row = seq * p.n + (static_cast<long long>(t) * p.R + r) * p.S + s;
         }
         const uint4* s_row = src + src_row * p.row_chunks;

@@ -1,5 +1,6 @@
 // skiparse_api.cu -- the C ABI of libskiparse.so (declared in include/skiparse.h):
-// argument validation, Skiparse-2D geometry, kernel launch and the per-device status word.
+// argument validation, Skiparse-2D and Skiparse-1D geometry, kernel launch and the per-device
+// status word.
 // Nothing here allocates device memory.
 #include <cuda_runtime.h>
 
@@ -30,34 +31,49 @@ constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
 int padded(int X, int P) { return ((X + P * P - 1) / (P * P)) * (P * P); }
 
-// Validates the shared shape arguments and fills the geometry. Returns a status code.
-int make_geometry(int B, int T, int H, int W, int heads, int d, int P, int mode, Geometry& g) {
+// Real (unpadded) positions of class c along an axis of X real positions with P classes: the
+// sub-grid positions whose coordinate (axis_coord) is below X. Token-wise the coordinates are
+// c, c+P, c+2P, ...; group-wise every full P^2 block gives each class P positions and the last,
+// partial block gives class c the part of [c*P, c*P+P) below X's remainder.
+int axis_real_count(int X, int c, int P, int mode) {
+    if (mode == SKIPARSE_TOKEN_WISE) return c < X ? (X - c + P - 1) / P : 0;
+    const int q = P * P, rem = X % q - c * P;
+    return (X / q) * P + (rem < 0 ? 0 : rem > P ? P : rem);
+}
+
+// Validates the shared shape arguments and fills the geometry of Skiparse-2D (dims 2) or
+// Skiparse-1D (dims 1). Returns a status code.
+int make_geometry(int dims, int B, int T, int H, int W, int heads, int d, int P, int mode,
+                  Geometry& g) {
     if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || P < 1) return SKIPARSE_ERR_INVALID_ARG;
     if (mode != SKIPARSE_TOKEN_WISE && mode != SKIPARSE_GROUP_WISE) return SKIPARSE_ERR_INVALID_ARG;
     if (P > skiparse::kMaxP) return SKIPARSE_ERR_UNSUPPORTED;
     if (d != 32 && d != 64 && d != 128) return SKIPARSE_ERR_UNSUPPORTED;
     const long long q2 = static_cast<long long>(P) * P;
     if (H > (1 << 24) || W > (1 << 24)) return SKIPARSE_ERR_UNSUPPORTED;
-    const long long Hp = (H + q2 - 1) / q2 * q2, Wp = (W + q2 - 1) / q2 * q2;
     const long long rows = static_cast<long long>(B) * T * H * W * heads;       // original rows
+    if (rows >= (1ll << 31)) return SKIPARSE_ERR_UNSUPPORTED;
+    // The frame axes the class rule runs on and the class count along each.
+    const long long Hax = dims == 2 ? H : 1, Wax = dims == 2 ? W : static_cast<long long>(H) * W;
+    const long long Ph = dims == 2 ? P : 1, Pw = dims == 2 ? P : q2;
+    const long long Hp = (Hax + Ph * Ph - 1) / (Ph * Ph) * (Ph * Ph);
+    const long long Wp = (Wax + Pw * Pw - 1) / (Pw * Pw) * (Pw * Pw);
     const long long prow = static_cast<long long>(B) * T * Hp * Wp * heads;     // rearranged rows
-    if (rows >= (1ll << 31) || prow >= (1ll << 31)) return SKIPARSE_ERR_UNSUPPORTED;
+    if (prow >= (1ll << 31)) return SKIPARSE_ERR_UNSUPPORTED;
     if (heads > 65535 || B * q2 > 65535) return SKIPARSE_ERR_UNSUPPORTED;
-    g.B = B; g.T = T; g.H = H; g.W = W; g.heads = heads; g.d = d; g.P = P; g.mode = mode;
+    g.B = B; g.T = T; g.heads = heads; g.d = d; g.P = P; g.mode = mode;
+    g.H = static_cast<int>(Hax);
+    g.W = static_cast<int>(Wax);
+    g.Ph = static_cast<int>(Ph);
+    g.Pw = static_cast<int>(Pw);
     g.Hp = static_cast<int>(Hp);
     g.Wp = static_cast<int>(Wp);
-    g.R = g.Hp / P;
-    g.S = g.Wp / P;
+    g.R = g.Hp / g.Ph;
+    g.S = g.Wp / g.Pw;
     g.n = static_cast<long long>(T) * g.R * g.S;
-    for (int c = 0; c < skiparse::kMaxP; ++c) {
-        g.Rc[c] = 0;
-        g.Sc[c] = 0;
-    }
-    for (int c = 0; c < P; ++c) {
-        for (int r = 0; r < g.R; ++r)
-            if (skiparse::axis_coord(r, c, P, mode) < H) ++g.Rc[c];
-        for (int s = 0; s < g.S; ++s)
-            if (skiparse::axis_coord(s, c, P, mode) < W) ++g.Sc[c];
+    for (int c = 0; c < skiparse::kMaxAxisClasses; ++c) {
+        g.Rc[c] = c < g.Ph ? axis_real_count(g.H, c, g.Ph, mode) : 0;
+        g.Sc[c] = c < g.Pw ? axis_real_count(g.W, c, g.Pw, mode) : 0;
     }
     return SKIPARSE_OK;
 }
@@ -112,14 +128,39 @@ long long skiparse_subseq_len(int T, int H, int W, int P) {
 
 long long skiparse_class_len(int T, int H, int W, int P, int mode, int ci, int cj) {
     Geometry g;
-    if (make_geometry(1, T, H, W, 1, 32, P, mode, g) != SKIPARSE_OK) return -1;
+    if (make_geometry(2, 1, T, H, W, 1, 32, P, mode, g) != SKIPARSE_OK) return -1;
     if (ci < 0 || cj < 0 || ci >= P || cj >= P) return -1;
     return static_cast<long long>(T) * g.Rc[ci] * g.Sc[cj];
 }
 
 long long skiparse_rearranged_numel(int B, int T, int H, int W, int heads, int d, int P) {
     Geometry g;
-    if (make_geometry(B, T, H, W, heads, d, P, SKIPARSE_TOKEN_WISE, g) != SKIPARSE_OK) return -1;
+    if (make_geometry(2, B, T, H, W, heads, d, P, SKIPARSE_TOKEN_WISE, g) != SKIPARSE_OK) return -1;
+    return static_cast<long long>(B) * P * P * g.n * heads * d;
+}
+
+long long skiparse1d_padded_length(long long L, int P) {
+    if (L < 1 || P < 1 || P > skiparse::kMaxP) return -1;
+    const long long q4 = static_cast<long long>(P) * P * P * P;
+    return (L + q4 - 1) / q4 * q4;
+}
+
+long long skiparse1d_subseq_len(int T, int H, int W, int P) {
+    Geometry g;
+    if (make_geometry(1, 1, T, H, W, 1, 32, P, SKIPARSE_TOKEN_WISE, g) != SKIPARSE_OK) return -1;
+    return g.n;
+}
+
+long long skiparse1d_class_len(int T, int H, int W, int P, int mode, int c) {
+    Geometry g;
+    if (make_geometry(1, 1, T, H, W, 1, 32, P, mode, g) != SKIPARSE_OK) return -1;
+    if (c < 0 || c >= P * P) return -1;
+    return static_cast<long long>(T) * g.Sc[c];
+}
+
+long long skiparse1d_rearranged_numel(int B, int T, int H, int W, int heads, int d, int P) {
+    Geometry g;
+    if (make_geometry(1, B, T, H, W, heads, d, P, SKIPARSE_TOKEN_WISE, g) != SKIPARSE_OK) return -1;
     return static_cast<long long>(B) * P * P * g.n * heads * d;
 }
 
@@ -164,28 +205,12 @@ int skiparse_get_device_status(skiparse_stream_t stream) {
     return v;
 }
 
-static int attn_fwd_common(const void* q, const void* k, const void* v, void* out, float* lse,
-                           int B, int T, int H, int W, int heads, int d, int P, int mode,
-                           skiparse_stream_t stream);
-
-int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int T,
-                        int H, int W, int heads, int d, int P, int mode, skiparse_stream_t stream) {
-    return attn_fwd_common(q, k, v, out, nullptr, B, T, H, W, heads, d, P, mode, stream);
-}
-
-int skiparse2d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
-                            int B, int T, int H, int W, int heads, int d, int P, int mode,
-                            skiparse_stream_t stream) {
-    if (!lse) return SKIPARSE_ERR_INVALID_ARG;
-    return attn_fwd_common(q, k, v, out, lse, B, T, H, W, heads, d, P, mode, stream);
-}
-
-static int attn_fwd_common(const void* q, const void* k, const void* v, void* out, float* lse,
-                           int B, int T, int H, int W, int heads, int d, int P, int mode,
-                           skiparse_stream_t stream) {
+static int attn_fwd_common(int dims, const void* q, const void* k, const void* v, void* out,
+                           float* lse, int B, int T, int H, int W, int heads, int d, int P,
+                           int mode, skiparse_stream_t stream) {
     if (!q || !k || !v || !out) return SKIPARSE_ERR_INVALID_ARG;
     Geometry g;
-    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    int st = make_geometry(dims, B, T, H, W, heads, d, P, mode, g);
     if (st != SKIPARSE_OK) return st;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SKIPARSE_ERR_MISALIGNED;
     const long long rows = static_cast<long long>(B) * T * H * W * heads;
@@ -207,8 +232,8 @@ static int attn_fwd_common(const void* q, const void* k, const void* v, void* ou
     p.lse = lse;
     p.status = status_ptr();
     if (!p.status) return SKIPARSE_ERR_CUDA;
-    p.T = T; p.H = H; p.W = W; p.heads = heads; p.P = P; p.mode = mode;
-    for (int c = 0; c < skiparse::kMaxP; ++c) {
+    p.T = T; p.H = g.H; p.W = g.W; p.heads = heads; p.Ph = g.Ph; p.Pw = g.Pw; p.mode = mode;
+    for (int c = 0; c < skiparse::kMaxAxisClasses; ++c) {
         p.Rc[c] = g.Rc[c];
         p.Sc[c] = g.Sc[c];
     }
@@ -219,13 +244,37 @@ static int attn_fwd_common(const void* q, const void* k, const void* v, void* ou
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
-int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
-                        const void* dout, const float* lse, void* dq, void* dk, void* dv, float* delta,
-                        int B, int T, int H, int W, int heads, int d, int P, int mode,
-                        skiparse_stream_t stream) {
+int skiparse2d_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int T,
+                        int H, int W, int heads, int d, int P, int mode, skiparse_stream_t stream) {
+    return attn_fwd_common(2, q, k, v, out, nullptr, B, T, H, W, heads, d, P, mode, stream);
+}
+
+int skiparse2d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int T, int H, int W, int heads, int d, int P, int mode,
+                            skiparse_stream_t stream) {
+    if (!lse) return SKIPARSE_ERR_INVALID_ARG;
+    return attn_fwd_common(2, q, k, v, out, lse, B, T, H, W, heads, d, P, mode, stream);
+}
+
+int skiparse1d_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int T,
+                        int H, int W, int heads, int d, int P, int mode, skiparse_stream_t stream) {
+    return attn_fwd_common(1, q, k, v, out, nullptr, B, T, H, W, heads, d, P, mode, stream);
+}
+
+int skiparse1d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int T, int H, int W, int heads, int d, int P, int mode,
+                            skiparse_stream_t stream) {
+    if (!lse) return SKIPARSE_ERR_INVALID_ARG;
+    return attn_fwd_common(1, q, k, v, out, lse, B, T, H, W, heads, d, P, mode, stream);
+}
+
+static int attn_bwd_common(int dims, const void* q, const void* k, const void* v, const void* out,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           float* delta, int B, int T, int H, int W, int heads, int d, int P,
+                           int mode, skiparse_stream_t stream) {
     if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta) return SKIPARSE_ERR_INVALID_ARG;
     Geometry g;
-    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    int st = make_geometry(dims, B, T, H, W, heads, d, P, mode, g);
     if (st != SKIPARSE_OK) return st;
     const void* bf[8] = {q, k, v, out, dout, dq, dk, dv};
     for (const void* ptr : bf)
@@ -257,8 +306,8 @@ int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void*
     p.dv = static_cast<uint16_t*>(dv);
     p.status = status_ptr();
     if (!p.status) return SKIPARSE_ERR_CUDA;
-    p.T = T; p.H = H; p.W = W; p.heads = heads; p.P = P; p.mode = mode;
-    for (int c = 0; c < skiparse::kMaxP; ++c) {
+    p.T = T; p.H = g.H; p.W = g.W; p.heads = heads; p.Ph = g.Ph; p.Pw = g.Pw; p.mode = mode;
+    for (int c = 0; c < skiparse::kMaxAxisClasses; ++c) {
         p.Rc[c] = g.Rc[c];
         p.Sc[c] = g.Sc[c];
     }
@@ -269,11 +318,27 @@ int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void*
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
-static int rearrange_common(const void* src, void* dst, int B, int T, int H, int W, int heads,
-                            int d, int P, int mode, skiparse_stream_t stream, int kind) {
+int skiparse2d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, float* delta,
+                        int B, int T, int H, int W, int heads, int d, int P, int mode,
+                        skiparse_stream_t stream) {
+    return attn_bwd_common(2, q, k, v, out, dout, lse, dq, dk, dv, delta, B, T, H, W, heads, d, P,
+                           mode, stream);
+}
+
+int skiparse1d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, float* delta,
+                        int B, int T, int H, int W, int heads, int d, int P, int mode,
+                        skiparse_stream_t stream) {
+    return attn_bwd_common(1, q, k, v, out, dout, lse, dq, dk, dv, delta, B, T, H, W, heads, d, P,
+                           mode, stream);
+}
+
+static int rearrange_common(int dims, const void* src, void* dst, int B, int T, int H, int W,
+                            int heads, int d, int P, int mode, skiparse_stream_t stream, int kind) {
     if (!src || !dst) return SKIPARSE_ERR_INVALID_ARG;
     Geometry g;
-    int st = make_geometry(B, T, H, W, heads, d, P, mode, g);
+    int st = make_geometry(dims, B, T, H, W, heads, d, P, mode, g);
     if (st != SKIPARSE_OK) return st;
     if (!aligned16(src) || !aligned16(dst)) return SKIPARSE_ERR_MISALIGNED;
     const long long row_bytes = static_cast<long long>(heads) * d * 2;
@@ -287,7 +352,8 @@ static int rearrange_common(const void* src, void* dst, int B, int T, int H, int
     skiparse::RearrangeParams p{};
     p.src = src;
     p.dst = dst;
-    p.B = B; p.T = T; p.H = H; p.W = W; p.P = P; p.mode = mode; p.R = g.R; p.S = g.S;
+    p.B = B; p.T = T; p.H = g.H; p.W = g.W; p.Ph = g.Ph; p.Pw = g.Pw; p.mode = mode;
+    p.R = g.R; p.S = g.S;
     p.n = g.n;
     p.row_chunks = static_cast<int>(row_bytes / 16);
     p.nrows = kind == 1 ? ntok : nslot;
@@ -297,17 +363,32 @@ static int rearrange_common(const void* src, void* dst, int B, int T, int H, int
 
 int skiparse_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d, int P,
                        int mode, skiparse_stream_t stream) {
-    return rearrange_common(x, y, B, T, H, W, heads, d, P, mode, stream, 0);
+    return rearrange_common(2, x, y, B, T, H, W, heads, d, P, mode, stream, 0);
 }
 
 int skiparse_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
                          int P, int mode, skiparse_stream_t stream) {
-    return rearrange_common(y, x, B, T, H, W, heads, d, P, mode, stream, 1);
+    return rearrange_common(2, y, x, B, T, H, W, heads, d, P, mode, stream, 1);
 }
 
 int skiparse_switch_mode(const void* y_src, void* y_dst, int B, int T, int H, int W, int heads,
                          int d, int P, int src_mode, skiparse_stream_t stream) {
-    return rearrange_common(y_src, y_dst, B, T, H, W, heads, d, P, src_mode, stream, 2);
+    return rearrange_common(2, y_src, y_dst, B, T, H, W, heads, d, P, src_mode, stream, 2);
+}
+
+int skiparse1d_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads, int d,
+                         int P, int mode, skiparse_stream_t stream) {
+    return rearrange_common(1, x, y, B, T, H, W, heads, d, P, mode, stream, 0);
+}
+
+int skiparse1d_unrearrange(const void* y, void* x, int B, int T, int H, int W, int heads, int d,
+                           int P, int mode, skiparse_stream_t stream) {
+    return rearrange_common(1, y, x, B, T, H, W, heads, d, P, mode, stream, 1);
+}
+
+int skiparse1d_switch_mode(const void* y_src, void* y_dst, int B, int T, int H, int W, int heads,
+                           int d, int P, int src_mode, skiparse_stream_t stream) {
+    return rearrange_common(1, y_src, y_dst, B, T, H, W, heads, d, P, src_mode, stream, 2);
 }
 
 }  // extern "C"

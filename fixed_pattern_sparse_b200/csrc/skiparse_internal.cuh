@@ -12,6 +12,12 @@
 // Because the coordinate map is increasing in the sub-grid position, the real (unpadded)
 // tokens of a class occupy a prefix [0, Rc) x [0, Sc) of its sub-grid; the kernels enumerate
 // only those, so the pad-key mask reduces to the ragged tail of the last key tile.
+//
+// Skiparse-1D (the flattened-sequence variant the summary page's 技术新颖性 and 实验结果
+// sections compare with) is the same one-axis rule on the in-frame index x = h*W + w with
+// ratio P^2. The kernels therefore take the class count of each axis separately: Skiparse-2D
+// runs on the (H, W) frame with (P, P) classes, Skiparse-1D on a (1, H*W) frame with
+// (1, P^2) classes; the rearranged layouts, the row maps and the launch grids are the same.
 #pragma once
 
 #include <cstdint>
@@ -19,6 +25,7 @@
 namespace skiparse {
 
 constexpr int kMaxP = 8;
+constexpr int kMaxAxisClasses = kMaxP * kMaxP;  // Skiparse-1D: P^2 classes on one axis
 
 // Spatial coordinate of sub-grid position `sub` of class `cls` along one axis.
 __host__ __device__ __forceinline__ int axis_coord(int sub, int cls, int P, int mode) {
@@ -37,12 +44,14 @@ __host__ __device__ __forceinline__ void axis_class(int x, int P, int mode, int&
 }
 
 struct Geometry {
-    int B, T, H, W, heads, d, P, mode;
-    int Hp, Wp;        // padded extents
-    int R, S;          // padded sub-grid extents Hp/P, Wp/P
+    int B, T, heads, d, P, mode;
+    int H, W;          // frame axes the class rule runs on: (H, W), or (1, H*W) for Skiparse-1D
+    int Ph, Pw;        // classes along each axis: (P, P), or (1, P^2) for Skiparse-1D
+    int Hp, Wp;        // padded extents (multiples of Ph^2 and Pw^2)
+    int R, S;          // padded sub-grid extents Hp/Ph, Wp/Pw
     long long n;       // padded subsequence length T*R*S
-    int Rc[kMaxP];     // real sub-grid rows of class row ci
-    int Sc[kMaxP];     // real sub-grid columns of class column cj
+    int Rc[kMaxAxisClasses];  // real sub-grid rows of class row ci
+    int Sc[kMaxAxisClasses];  // real sub-grid columns of class column cj
 };
 
 // Parameters of the fused attention kernel.
@@ -53,8 +62,8 @@ struct AttnParams {
     uint16_t* out;
     float* lse;                    // optional (nullptr): log-sum-exp of q.k/sqrt(d) per (token, head)
     int* status;                   // device error word
-    int T, H, W, heads, P, mode;
-    int Rc[kMaxP], Sc[kMaxP];
+    int T, H, W, heads, Ph, Pw, mode;  // H, W, Ph, Pw as in Geometry
+    int Rc[kMaxAxisClasses], Sc[kMaxAxisClasses];
     float scale_log2;              // log2(e)/sqrt(d)
     unsigned long long wait_limit_ns;
     int fault;                     // test hook: 1 = one producer never signals the first K tile
@@ -73,8 +82,8 @@ struct BwdParams {
     uint16_t* dk;
     uint16_t* dv;
     int* status;
-    int T, H, W, heads, P, mode;
-    int Rc[kMaxP], Sc[kMaxP];
+    int T, H, W, heads, Ph, Pw, mode;  // H, W, Ph, Pw as in Geometry
+    int Rc[kMaxAxisClasses], Sc[kMaxAxisClasses];
     float scale_log2;              // log2(e)/sqrt(d)
     float scale;                   // 1/sqrt(d)
     unsigned long long wait_limit_ns;
@@ -83,7 +92,7 @@ struct BwdParams {
 struct RearrangeParams {
     const void* src;
     void* dst;
-    int B, T, H, W, P, mode, R, S;
+    int B, T, H, W, Ph, Pw, mode, R, S;  // H, W, Ph, Pw as in Geometry
     long long n;          // padded subsequence length
     int row_chunks;       // 16-byte chunks per token row (heads*d*2/16)
     long long nrows;      // rows to write: B*P*P*n (rearrange, switch) or B*T*H*W (unrearrange)

@@ -1,5 +1,6 @@
 /*
- * skiparse.h -- C ABI of libskiparse.so: Skiparse-2D sparse attention on NVIDIA B200 (sm_100a).
+ * skiparse.h -- C ABI of libskiparse.so: Skiparse-2D (and Skiparse-1D) sparse attention on
+ * NVIDIA B200 (sm_100a).
  *
  * The method (paper.rainbus.top summary of "OSP-Next: Efficient High-Quality Video Generation
  * with Sparse Sequence Parallelism, HiF8 Quantization, and Reinforcement Learning", sections
@@ -166,6 +167,53 @@ SKIPARSE_API long long skiparse_subseq_len(int T, int H, int W, int P);
 
 /* Number of real tokens of class (ci, cj) in one batch element; -1 on invalid arguments. */
 SKIPARSE_API long long skiparse_class_len(int T, int H, int W, int P, int mode, int ci, int cj);
+
+/*
+ * ---- Skiparse-1D ------------------------------------------------------------------------
+ * The 1D skip pattern on the flattened sequence, the variant that the summary page's sections
+ * 技术新颖性 (novelty) and 实验结果 (results) compare Skiparse-2D with; the pages give no formula
+ * for it. The reading implemented here: the in-frame index x = h*W + w with ratio P^2, so that
+ * there are P^2 subsequences as in Skiparse-2D --
+ *   token-wise class x mod P^2,              position in the class x div P^2;
+ *   group-wise class (x div P^2) mod P^2,    position (x div P^4)*P^2 + x mod P^2
+ *   (runs of P^2 consecutive tokens stay together);
+ * each frame's H*W positions are padded at the end to Lp, the next multiple of P^4, and the
+ * padded keys are masked. Rearranged layout: (B*P*P, n, heads, d) with n = T * Lp / P^2,
+ * subsequence b*P^2 + class, tokens in (t, position-in-class) order.
+ * Every function below takes the same arguments, with the same layout, ownership, alignment,
+ * aliasing and error rules, as the Skiparse-2D function of the same name; only the class rule
+ * differs. Supported sizes as above (1 <= P <= 8; B*T*Lp*heads < 2^31).
+ */
+SKIPARSE_API int skiparse1d_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                     int B, int T, int H, int W, int heads, int d, int P, int mode,
+                                     skiparse_stream_t stream);
+SKIPARSE_API int skiparse1d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out,
+                                         float* lse, int B, int T, int H, int W, int heads, int d,
+                                         int P, int mode, skiparse_stream_t stream);
+SKIPARSE_API int skiparse1d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                     const void* dout, const float* lse, void* dq, void* dk,
+                                     void* dv, float* delta, int B, int T, int H, int W, int heads,
+                                     int d, int P, int mode, skiparse_stream_t stream);
+/* x (B,T,H,W,heads,d) -> y (B*P*P, n, heads, d), pad slots +0.0; bit-exact row permutation. */
+SKIPARSE_API int skiparse1d_rearrange(const void* x, void* y, int B, int T, int H, int W, int heads,
+                                      int d, int P, int mode, skiparse_stream_t stream);
+/* y (B*P*P, n, heads, d) -> x (B,T,H,W,heads,d); pad slots ignored. */
+SKIPARSE_API int skiparse1d_unrearrange(const void* y, void* x, int B, int T, int H, int W,
+                                        int heads, int d, int P, int mode,
+                                        skiparse_stream_t stream);
+/* src_mode's Skiparse-1D rearranged layout -> the other mode's, in one pass; pad slots +0.0. */
+SKIPARSE_API int skiparse1d_switch_mode(const void* y_src, void* y_dst, int B, int T, int H,
+                                        int W, int heads, int d, int P, int src_mode,
+                                        skiparse_stream_t stream);
+/* Per-frame length L padded to the next multiple of P^4; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse1d_padded_length(long long L, int P);
+/* Padded subsequence length n = T * Lp / P^2; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse1d_subseq_len(int T, int H, int W, int P);
+/* Real tokens of class c (0 <= c < P^2) in one batch element; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse1d_class_len(int T, int H, int W, int P, int mode, int c);
+/* Elements of the Skiparse-1D rearranged tensor, B*P*P*n*heads*d; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse1d_rearranged_numel(int B, int T, int H, int W, int heads, int d,
+                                                   int P);
 
 /*
  * Synchronizes `stream`, then returns and clears the current device's error word: SKIPARSE_OK,

@@ -57,3 +57,17 @@ def sample_rows_one_class(w, mode: int, count: int, cls: int = 0, head: int = 0,
     rng = np.random.default_rng(seed)
     pick = np.unique(np.concatenate([toks[:2], toks[-2:], rng.choice(toks, size=min(count, len(toks)), replace=False)]))
     return pick.astype(np.int64) * w.heads + head
+
+
+def sample_rows_one_class_1d(w, mode: int, count: int, cls: int = 0, head: int = 0, seed: int = 0) -> np.ndarray:
+    """sample_rows_one_class for Skiparse-1D: the class of in-frame index x = h*W + w from the
+    brute force's own restatement of the 1D rule."""
+    from oracle import brute
+    k2 = (w.P * w.P) ** 2
+    L = w.H * w.W
+    Lp = -(-L // k2) * k2
+    xs = np.nonzero(brute.class_1d(Lp, w.P, mode)[:L] == cls)[0]
+    toks = (np.arange(w.T)[:, None] * L + xs[None, :]).reshape(-1)
+    rng = np.random.default_rng(seed)
+    pick = np.unique(np.concatenate([toks[:2], toks[-2:], rng.choice(toks, size=min(count, len(toks)), replace=False)]))
+    return pick.astype(np.int64) * w.heads + head

@@ -80,6 +80,40 @@ def test_geometry_matches_oracle(L):
         assert n == 2 * P * P * oracle.subseq_len(T, H, W, P) * 3 * 64
 
 
+def test_geometry_1d_matches_oracle(L):
+    """Skiparse-1D: padded length, subsequence length and real per-class counts of the product's
+    geometry against the oracle's 1D rearrange."""
+    import numpy as np
+    for L_, P in [(1, 2), (15, 2), (16, 2), (17, 2), (3600, 2), (1560, 2), (81, 3), (4032, 8), (5, 1)]:
+        assert L.skiparse1d_padded_length(L_, P) == oracle.padded_length_1d(L_, P)
+    for (T, H, W, P) in [(2, 8, 8, 2), (3, 10, 14, 2), (1, 5, 7, 3), (2, 3, 20, 4), (1, 45, 80, 2),
+                         (1, 30, 52, 2), (2, 6, 5, 1), (1, 1, 1, 2)]:
+        assert L.skiparse1d_subseq_len(T, H, W, P) == oracle.subseq_len(T, H, W, P, dims=1)
+        for mode in (0, 1):
+            x = (np.arange(T * H * W, dtype=np.uint16) + 1).reshape(1, T, H, W, 1, 1)
+            y = oracle.rearrange(x, P, mode, dims=1)
+            for c in range(P * P):
+                real = int((y[c, :, 0, 0] > 0).sum())
+                assert L.skiparse1d_class_len(T, H, W, P, mode, c) == real
+            assert L.skiparse1d_class_len(T, H, W, P, mode, P * P) == -1
+        n = L.skiparse1d_rearranged_numel(2, T, H, W, 3, 64, P)
+        assert n == 2 * P * P * oracle.subseq_len(T, H, W, P, dims=1) * 3 * 64
+
+
+def test_1d_entries_reject_bad_arguments_synchronously(L):
+    assert L.skiparse1d_attn_fwd(0, FAKE, FAKE, FAKE + 4096, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
+    assert L.skiparse1d_attn_fwd(FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 32, 9, 0, None) == 2
+    assert L.skiparse1d_attn_fwd(FAKE, FAKE, FAKE, FAKE + (1 << 20), 1, 2, 8, 8, 2, 32, 2, 3, None) == 1
+    assert L.skiparse1d_attn_fwd_lse(FAKE, FAKE, FAKE, FAKE + (1 << 20), 0, 1, 2, 8, 8, 2, 32, 2, 0,
+                                     None) == 1
+    assert L.skiparse1d_attn_bwd(*([FAKE] * 9), 0, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
+    assert L.skiparse1d_rearrange(FAKE, FAKE + 4, 1, 2, 8, 8, 2, 32, 2, 0, None) == 3
+    assert L.skiparse1d_unrearrange(FAKE, FAKE + 64, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
+    assert L.skiparse1d_switch_mode(FAKE, FAKE, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
+    # padded rows past 2^31: 1D pads each frame to a multiple of P^4 = 4096
+    assert L.skiparse1d_rearrange(FAKE, FAKE + (1 << 40), 1, 1 << 16, 1, 1, 8192, 32, 8, 0, None) == 2
+
+
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails before any CUDA call
 
 
