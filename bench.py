@@ -49,6 +49,8 @@ KNOWN_TRAFFIC = {
     # the 720p launch by the ratio of token rows (7.692); traffic grows with q/k/v/out because the
     # kernel reads each input once and writes the output once.
     "2a906497c379c4ad": 2.955e9,
+    # the per-axis class-count kernel: 480p capture 302.5 + 80.1 MB per launch, x 7.692
+    "726002548e064429": 2.943e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
