@@ -63,16 +63,15 @@ struct BwdCfg : TileGeom<D> {
 // rows 64..127 -> columns 64..95.
 __device__ __forceinline__ uint32_t half_packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
 
-// 4-byte cp.async of one fp32 per tile row (L or D of the row's token and head).
-__device__ __forceinline__ void load_vec(uint32_t dst, const float* __restrict__ src, const RowMap& rows,
-                                         int first, int n_c, int pw, int lane) {
+// 4-byte cp.async of one fp32 per tile row (L or D of the row's token and head); tr holds the
+// token rows of this lane's two tile rows 64*pw + lane and 64*pw + 32 + lane.
+__device__ __forceinline__ void load_vec(uint32_t dst, const float* __restrict__ src, const TileRows& tr,
+                                         int pw, int lane) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int r = 64 * pw + 32 * half + lane;
-        int i = first + r;
-        i = i < n_c ? i : n_c - 1;
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst + 4u * r),
-                     "l"(src + rows(i))
+                     "l"(src + (half ? tr.rb : tr.ra))
                      : "memory");
     }
 }
@@ -90,7 +89,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
     const int first = tile * kTileRows;
     if (first >= n_c) return;  // uniform over the CTA, before any shared state
     const int nstream = (n_c + kTileRows - 1) / kTileRows;
-    const RowMap rows{p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head};
+    RowMap rows;
+    rows.init(p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = ptx::smem_u32(smem_raw);
@@ -139,11 +139,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
     if (warp == kBwdProd0 || warp == kBwdProd0 + 1) {
         // ------------------------------------------------------------------ producers
         const int pw = warp - kBwdProd0;
-        load_tile<D>(sbase + C::OFF_A1, g_a1, rows, first, n_c, pw, lane);
-        load_tile<D>(sbase + C::OFF_A2, g_a2, rows, first, n_c, pw, lane);
+        const TileRows ta = tile_rows(rows, first, n_c, pw, lane);
+        load_tile_rows<D>(sbase + C::OFF_A1, g_a1, ta, pw, lane);
+        load_tile_rows<D>(sbase + C::OFF_A2, g_a2, ta, pw, lane);
         if (!KV) {  // the stationary queries' L and D
-            load_vec(sbase + C::OFF_VEC, p.lse, rows, first, n_c, pw, lane);
-            load_vec(sbase + C::OFF_VEC + 4 * kTileRows, p.delta, rows, first, n_c, pw, lane);
+            load_vec(sbase + C::OFF_VEC, p.lse, ta, pw, lane);
+            load_vec(sbase + C::OFF_VEC + 4 * kTileRows, p.delta, ta, pw, lane);
         }
         cp_async_commit();
         uint32_t prev_bar = bar(C::B_STAT);
@@ -160,12 +161,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 }
             }
             const uint32_t slot = sbase + C::OFF_B + 2 * s * C::TILE_BYTES;
-            load_tile<D>(slot, g_b1, rows, j * kTileRows, n_c, pw, lane);
-            load_tile<D>(slot + C::TILE_BYTES, g_b2, rows, j * kTileRows, n_c, pw, lane);
+            const TileRows tr = tile_rows(rows, j * kTileRows, n_c, pw, lane);
+            load_tile_rows<D>(slot, g_b1, tr, pw, lane);
+            load_tile_rows<D>(slot + C::TILE_BYTES, g_b2, tr, pw, lane);
             if (KV) {  // the streamed queries' L and D
                 const uint32_t v = sbase + C::OFF_VEC + s * 2 * 4 * kTileRows;
-                load_vec(v, p.lse, rows, j * kTileRows, n_c, pw, lane);
-                load_vec(v + 4 * kTileRows, p.delta, rows, j * kTileRows, n_c, pw, lane);
+                load_vec(v, p.lse, tr, pw, lane);
+                load_vec(v + 4 * kTileRows, p.delta, tr, pw, lane);
             }
             cp_async_commit();
             cp_async_wait<1>();

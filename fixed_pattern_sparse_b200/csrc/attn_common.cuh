@@ -31,17 +31,54 @@ struct TileGeom {
     static constexpr uint32_t kstep_off(int kk) { return (kk / KPB) * BOX_BYTES + (kk % KPB) * 32; }
 };
 
+// Division by a divisor that is fixed for a whole CTA, as one multiply-high, an add and a shift
+// (T. Granlund and P. Montgomery, "Division by invariant integers using multiplication",
+// PLDI 1994): for d >= 1 and 0 <= n < 2^31, n div d = (umulhi(n, m) + n) >> l with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1 (umulhi(n, m) < n, so the sum fits
+// 32 bits). The producers evaluate the class-local -> token row map for every row they load;
+// with runtime divisions it cost them more issue slots than the copies themselves.
+struct FastDiv {
+    uint32_t m;
+    uint32_t l;
+    __host__ __device__ void init(int d) {
+        const uint32_t dd = d < 1 ? 1u : static_cast<uint32_t>(d);
+        l = 0;
+        while ((1ull << l) < dd) ++l;
+        m = static_cast<uint32_t>((((1ull << 32) * ((1ull << l) - dd)) / dd) + 1);
+    }
+    __device__ __forceinline__ int div(int n) const {
+        return static_cast<int>((__umulhi(static_cast<uint32_t>(n), m) + static_cast<uint32_t>(n)) >> l);
+    }
+};
+
 // Global row (token*heads + head) of the class-local real token i of (b, ci, cj).
 struct RowMap {
     int T, H, W, heads, Ph, Pw, mode;
     int ci, cj, Rc, Sc, b, head;
+    FastDiv dSc, dRc, dPh, dPw;
+    __device__ __forceinline__ void init(int T_, int H_, int W_, int heads_, int Ph_, int Pw_,
+                                         int mode_, int ci_, int cj_, int Rc_, int Sc_, int b_,
+                                         int head_) {
+        T = T_; H = H_; W = W_; heads = heads_; Ph = Ph_; Pw = Pw_; mode = mode_;
+        ci = ci_; cj = cj_; Rc = Rc_; Sc = Sc_; b = b_; head = head_;
+        dSc.init(Sc);
+        dRc.init(Rc);
+        dPh.init(Ph);
+        dPw.init(Pw);
+    }
+    // axis_coord (skiparse_internal.cuh) with the group-wise division by P done as above
+    __device__ __forceinline__ int coord(int sub, int cls, int P, const FastDiv& dP) const {
+        if (mode == 0) return cls + P * sub;
+        const int blk = dP.div(sub);
+        return blk * P * P + cls * P + (sub - blk * P);
+    }
     __device__ __forceinline__ int operator()(int i) const {
-        const int s = i % Sc;
-        const int tr = i / Sc;
-        const int r = tr % Rc;
-        const int t = tr / Rc;
-        const int h = axis_coord(r, ci, Ph, mode);
-        const int w = axis_coord(s, cj, Pw, mode);
+        const int tr = dSc.div(i);
+        const int s = i - tr * Sc;
+        const int t = dRc.div(tr);
+        const int r = tr - t * Rc;
+        const int h = coord(r, ci, Ph, dPh);
+        const int w = coord(s, cj, Pw, dPw);
         return (((b * T + t) * H + h) * W + w) * heads + head;
     }
 };
@@ -61,22 +98,30 @@ __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Issues the cp.async copies of tile rows [first, first+128) of the class's real-token list
-// (rows past n_c repeat row n_c-1; they are masked or never stored) into a 128-row tile laid
-// out as the UMMA canonical K-major layout with 128-byte (64-byte for d = 32) swizzle.
-// Producer warp pw (0/1) copies tile rows [64*pw, 64*pw+64); 16 consecutive lanes cover one
-// 256-byte row so every warp instruction reads whole rows.
+// The two token rows a producer lane copies for tile rows [first, first+128) of the class's
+// real-token list: tile rows 64*pw + lane and 64*pw + lane + 32 (rows past n_c repeat row
+// n_c-1; they are masked or never stored). K and V tiles of one key step share them.
+struct TileRows {
+    int ra, rb;
+};
+__device__ __forceinline__ TileRows tile_rows(const RowMap& rows, int first, int n_c, int pw, int lane) {
+    int ia = first + 64 * pw + lane, ib = ia + 32;
+    ia = ia < n_c ? ia : n_c - 1;
+    ib = ib < n_c ? ib : n_c - 1;
+    return TileRows{rows(ia), rows(ib)};
+}
+
+// Issues the cp.async copies of a 128-row tile whose token rows tile_rows() gave into the
+// UMMA canonical K-major layout with 128-byte (64-byte for d = 32) swizzle. Producer warp pw
+// (0/1) copies tile rows [64*pw, 64*pw+64); 16 consecutive lanes cover one 256-byte row so
+// every warp instruction reads whole rows.
 template <int D>
-__device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restrict__ g,
-                                          const RowMap& rows, int first, int n_c, int pw, int lane) {
+__device__ __forceinline__ void load_tile_rows(uint32_t dst, const uint16_t* __restrict__ g,
+                                               const TileRows& tr, int pw, int lane) {
     using C = TileGeom<D>;
     constexpr int CPR = D * 2 / 16;   // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;     // rows per warp instruction
     constexpr int NI = 64 / RPI;      // warp instructions per producer warp
-    int ia = first + 64 * pw + lane, ib = ia + 32;
-    ia = ia < n_c ? ia : n_c - 1;
-    ib = ib < n_c ? ib : n_c - 1;
-    const int ra = rows(ia), rb = rows(ib);
     const int c = lane % CPR;
     const int rsub = lane / CPR;
     const uint32_t box = static_cast<uint32_t>((c * 16) / C::SW);
@@ -84,13 +129,20 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restri
 #pragma unroll
     for (int k = 0; k < NI; ++k) {
         const int rl = k * RPI + rsub;  // 0..63
-        const int grow = __shfl_sync(0xffffffffu, (k * RPI < 32) ? ra : rb, rl & 31);
+        const int grow = __shfl_sync(0xffffffffu, (k * RPI < 32) ? tr.ra : tr.rb, rl & 31);
         const int r = 64 * pw + rl;     // tile row 0..127
         const uint32_t sw = C::SW == 128 ? (cb ^ static_cast<uint32_t>(r & 7))
                                          : (cb ^ static_cast<uint32_t>((r >> 1) & 3));
         const uint32_t d = dst + box * C::BOX_BYTES + static_cast<uint32_t>(r) * C::SW + sw * 16u;
         cp_async_16(d, g + static_cast<size_t>(grow) * D + c * 8);
     }
+}
+
+// tile_rows + load_tile_rows for a tile loaded from one tensor only.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restrict__ g,
+                                          const RowMap& rows, int first, int n_c, int pw, int lane) {
+    load_tile_rows<D>(dst, g, tile_rows(rows, first, n_c, pw, lane), pw, lane);
 }
 
 

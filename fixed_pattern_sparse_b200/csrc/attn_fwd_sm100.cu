@@ -129,7 +129,8 @@ __device__ __forceinline__ float exp_chunk(const uint32_t* v, float sl2, float n
         const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sl2, neg);
         float p0, p1;
         if (EMU && (kEmuMask & (1u << e))) {
-            ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), p0, p1);
+            p0 = ptx::exp2_poly(x0);
+            p1 = ptx::exp2_poly(x1);
         } else {
             p0 = ptx::ex2_approx(x0);
             p1 = ptx::ex2_approx(x1);
@@ -155,7 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
     const int q_first = pair * 2 * kBM;
     if (q_first >= n_c) return;  // uniform over the CTA, before any shared state
     const int nkv = (n_c + kBN - 1) / kBN;
-    const RowMap rows{p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head};
+    RowMap rows;
+    rows.init(p.T, p.H, p.W, p.heads, p.Ph, p.Pw, p.mode, ci, cj, Rc, Sc, b, head);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = ptx::smem_u32(smem_raw);
@@ -215,11 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         cp_async_commit();
         uint32_t prev_bar = bar(C::B_Q);
         bool ok = true;
+        TileRows kv{0, 0};  // token rows of key step j, shared by its K and V tiles
         for (int L = 0; L < 2 * nkv; ++L) {
             const int j = L >> 1;
             const bool is_v = L & 1;
             const int nst = is_v ? C::VST : C::KST;
             const int s = j % nst;
+            if (!is_v) kv = tile_rows(rows, j * kBN, n_c, pw, lane);
             if (j >= nst) {
                 const int empty = (is_v ? C::B_VEMPTY : C::B_KEMPTY) + s;
                 int w_ok = 1;
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 }
             }
             const uint32_t dst = sbase + (is_v ? C::OFF_V : C::OFF_K) + s * C::TILE_BYTES;
-            load_tile<D>(dst, is_v ? p.v : p.k, rows, j * kBN, n_c, pw, lane);
+            load_tile_rows<D>(dst, is_v ? p.v : p.k, kv, pw, lane);
             cp_async_commit();
             cp_async_wait<1>();   // the previous load has landed
             fence_proxy_async();  // make it visible to the tensor core (async proxy)
@@ -359,26 +363,30 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 // tile sets the reference max; the ragged last tile has masked keys).
                 float sc[kBN];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
+                for (int g = 0; g < 4; ++g)
                     ptx::tmem_ld32(s_addr + 32 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * g]));
-                    ptx::tmem_wait_ld();
+                ptx::tmem_wait_ld();  // one wait for the whole 128-column row
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sc[32 * g + e] = __uint_as_float(sv[32 * g + e]);
-                }
+                for (int e = 0; e < kBN; ++e) sc[e] = __uint_as_float(sv[e]);
                 if (last) {
                     const int valid = n_c - j * kBN;
 #pragma unroll
                     for (int e = 0; e < kBN; ++e)
                         if (e >= valid) sc[e] = -INFINITY;
                 }
-                float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
+                // row max with 3-input max instructions, four independent chains
+                float mx0 = ptx::max3f(sc[0], sc[1], sc[2]), mx1 = ptx::max3f(sc[3], sc[4], sc[5]);
+                float mx2 = ptx::max3f(sc[6], sc[7], sc[8]), mx3 = ptx::max3f(sc[9], sc[10], sc[11]);
 #pragma unroll
-                for (int e = 4; e < kBN; e += 4) {
-                    mx0 = fmaxf(mx0, sc[e]);
-                    mx1 = fmaxf(mx1, sc[e + 1]);
-                    mx2 = fmaxf(mx2, sc[e + 2]);
-                    mx3 = fmaxf(mx3, sc[e + 3]);
+                for (int e = 12; e + 8 <= kBN; e += 8) {
+                    mx0 = ptx::max3f(mx0, sc[e], sc[e + 1]);
+                    mx1 = ptx::max3f(mx1, sc[e + 2], sc[e + 3]);
+                    mx2 = ptx::max3f(mx2, sc[e + 4], sc[e + 5]);
+                    mx3 = ptx::max3f(mx3, sc[e + 6], sc[e + 7]);
                 }
+                static_assert((kBN - 12) % 8 == 4, "tail of the max chains");
+                mx0 = ptx::max3f(mx0, sc[kBN - 4], sc[kBN - 3]);
+                mx1 = ptx::max3f(mx1, sc[kBN - 2], sc[kBN - 1]);
                 const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 if (j == 0 || mx > m_run + thresh) {
                     alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
@@ -399,7 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                         const float x1 = fmaf(sc[32 * g + 2 * e + 1], sl2, neg);
                         float p0, p1;
                         if (kEmuMask != 0u && !last && (kEmuMask & (1u << e))) {
-                            ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), p0, p1);
+                            p0 = ptx::exp2_poly(x0);
+                            p1 = ptx::exp2_poly(x1);
                         } else {
                             p0 = ptx::ex2_approx(x0);
                             p1 = ptx::ex2_approx(x1);
@@ -547,7 +556,8 @@ __global__ void skiparse_exp2_kernel(const float* __restrict__ x, float* __restr
     const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
     float y0, y1;
     if (method == 1) {
-        ptx::f2_unpack(ptx::exp2_poly_f2(ptx::f2_pack(x0, x1)), y0, y1);
+        y0 = ptx::exp2_poly(x0);
+        y1 = ptx::exp2_poly(x1);
     } else {
         y0 = ptx::ex2_approx(x0);
         y1 = ptx::ex2_approx(x1);

@@ -302,24 +302,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // relative error) and give max relative error 7.5e-5 in fp32 Horner form, 26x below half an
 // ulp of bf16, the precision P is kept in. x is clamped at -125 so the exponent field cannot
 // underflow (2^-125 ~ 2.4e-38 stands in for smaller results).
-__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
-    const uint64_t magic = f2_pack(12582912.f, 12582912.f);     // 1.5 * 2^23
-    const uint64_t t = f2_add(f2_pack(x0, x1), magic);           // round(x) in the low bits
-    const uint64_t nf = f2_add(t, f2_pack(-12582912.f, -12582912.f));
-    const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), f2_pack(x0, x1));
-    uint64_t p = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.242611125f, 0.242611125f));
-    p = f2_fma(p, f, f2_pack(0.693260968f, 0.693260968f));
-    p = f2_fma(p, f, f2_pack(0.999928057f, 0.999928057f));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    const uint32_t r0 = __float_as_uint(t0) * 8388608u + __float_as_uint(p0);  // n << 23 added
-    const uint32_t r1 = __float_as_uint(t1) * 8388608u + __float_as_uint(p1);
-    return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);                             // keeps n + 127 inside the exponent field
+    const float t = x + 12582912.f;                   // 1.5 * 2^23: round(x) in the low bits
+    const float f = x - (t - 12582912.f);             // f in [-1/2, 1/2]
+    float p = fmaf(0.0551716685f, f, 0.242611125f);
+    p = fmaf(p, f, 0.693260968f);
+    p = fmaf(p, f, 0.999928057f);
+    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));  // n << 23 added
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
