@@ -18,12 +18,14 @@
 // P_i (bf16 pairs) is written over the first 64 columns of S_i and is the A operand of
 // O_i += P_i * V straight from TMEM. MMA order per key tile j:
 //   O0 += P0(j) V_j ; S0(j+1) = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1(j+1) = Q1 K_{j+1}^T
-// so the softmax of one query tile overlaps the tensor-core work of the other.
+// so the softmax of one query tile overlaps the tensor-core work of the other. The softmax
+// releases P in two halves of the key tile, and O += P V on the first half starts while the
+// exponentials of the second half run.
 // Softmax rescales O lazily: only when a row maximum grows by more than 2^8 (FlashAttention-4's
 // lazy rescaling); the stale maximum keeps every p <= 256, exact after the final division.
 // Options (compile-time, off by default because they measured no faster on B200): MUFU turns
-// between the two softmax warpgroups, exponentials against a stale running max, part of the
-// exponentials as a polynomial on the FMA pipe (a FlashAttention-4 idea), a setmaxnreg split.
+// between the two softmax warpgroups, part of the exponentials as a polynomial on the FMA pipe
+// (a FlashAttention-4 idea), a setmaxnreg split.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -39,14 +41,10 @@ constexpr int kBN = 128;   // keys per tile
 #ifndef SKIPARSE_REGSPLIT
 #define SKIPARSE_REGSPLIT 0
 #endif
-// Optional softmax schedules, measured no faster on B200 and therefore off by default:
-// MUFU turns (the two softmax warpgroups take turns on the exponential unit) and stale-max
-// exponentials (taken against the running max while the next chunk of S loads).
+// Optional softmax schedule, measured no faster on B200 and therefore off by default: MUFU
+// turns (the two softmax warpgroups take turns on the exponential unit).
 #ifndef SKIPARSE_MUFU_TURNS
 #define SKIPARSE_MUFU_TURNS 0
-#endif
-#ifndef SKIPARSE_STALE_MAX
-#define SKIPARSE_STALE_MAX 0
 #endif
 constexpr int kThreads = SKIPARSE_REGSPLIT ? 384 : 352;
 constexpr int kLaunchRegs = 168;       // 65536 / 384 rounded down to a multiple of 8
@@ -87,8 +85,8 @@ struct Cfg : TileGeom<D> {
     static constexpr int B_VFULL = B_KEMPTY + KST;
     static constexpr int B_VEMPTY = B_VFULL + VST;
     static constexpr int B_SFULL = B_VEMPTY + VST;        // 2: one per query tile
-    static constexpr int B_PFULL = B_SFULL + 2;           // 2
-    static constexpr int B_TURN = B_PFULL + 2;            // 2: MUFU turn of query tile 0 / 1
+    static constexpr int B_PFULL = B_SFULL + 2;           // 4: (query tile, half of the key tile)
+    static constexpr int B_TURN = B_PFULL + 4;            // 2: MUFU turn of query tile 0 / 1
     static constexpr int B_OFULL = B_TURN + 2;
     static constexpr int B_DRAIN = B_OFULL + 1;
     static constexpr int NBARS = B_DRAIN + 1;
@@ -101,47 +99,6 @@ struct Cfg : TileGeom<D> {
     static_assert(COL_O1 + D <= NCOLS, "TMEM overflow");
     static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
 };
-
-template <int N>
-__device__ __forceinline__ float row_max(const uint32_t* v) {
-    float m0 = __uint_as_float(v[0]), m1 = __uint_as_float(v[1]);
-    float m2 = __uint_as_float(v[2]), m3 = __uint_as_float(v[3]);
-#pragma unroll
-    for (int e = 4; e < N; e += 4) {
-        m0 = fmaxf(m0, __uint_as_float(v[e]));
-        m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
-        m2 = fmaxf(m2, __uint_as_float(v[e + 2]));
-        m3 = fmaxf(m3, __uint_as_float(v[e + 3]));
-    }
-    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-}
-
-// p = 2^(s*sl2 + neg) for 32 scores; the bf16 pairs go to 16 TMEM columns at p_addr (over the
-// scores already read). EMU selects the column pairs of kEmuMask for the FMA-pipe polynomial.
-// Returns the fp32 sum of the 32 probabilities.
-template <bool EMU>
-__device__ __forceinline__ float exp_chunk(const uint32_t* v, float sl2, float neg, uint32_t p_addr) {
-    uint32_t pk[16];
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const float x0 = fmaf(__uint_as_float(v[2 * e]), sl2, neg);
-        const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), sl2, neg);
-        float p0, p1;
-        if (EMU && (kEmuMask & (1u << e))) {
-            p0 = ptx::exp2_poly(x0);
-            p1 = ptx::exp2_poly(x1);
-        } else {
-            p0 = ptx::ex2_approx(x0);
-            p1 = ptx::ex2_approx(x1);
-        }
-        s0 += p0;
-        s1 += p1;
-        pk[e] = ptx::pack_bf16x2(p0, p1);
-    }
-    ptx::tmem_st16(p_addr, pk);
-    return s0 + s1;
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const AttnParams p) {
@@ -184,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
-            ptx::mbar_init(bar(C::B_PFULL + i), kBM);
+            ptx::mbar_init(bar(C::B_PFULL + 2 * i), kBM);
+            ptx::mbar_init(bar(C::B_PFULL + 2 * i + 1), kBM);
             ptx::mbar_init(bar(C::B_TURN + i), kBM);
         }
         ptx::mbar_init(bar(C::B_OFULL), 1);
@@ -268,12 +226,26 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     ptx::mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_o = [&](uint32_t p_tmem, int vslot, uint32_t d_tmem, bool acc) {
+            // O += P V over one half of the key tile (keys [64h, 64h+64)), as soon as the softmax
+            // has released that half of P
+            auto issue_o_half = [&](uint32_t p_tmem, int vslot, uint32_t d_tmem, bool acc, int h) {
                 const uint64_t vd = vd0 + ((vslot * C::TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
+                for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                    const int kk = h * (kBN / 32) + k4;
                     ptx::mma_ts(d_tmem, p_tmem + kk * 8, vd + ((kk * 16 * C::SW) >> 4), idesc_o,
                                 (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            auto issue_o = [&](int qt, int vslot, bool acc, int phase) -> bool {
+                const uint32_t p_tmem = tmem + (qt ? C::COL_S1 : C::COL_S0);
+                const uint32_t d_tmem = tmem + (qt ? C::COL_O1 : C::COL_O0);
+                for (int h = 0; h < 2; ++h) {
+                    if (!ptx::mbar_wait(bar(C::B_PFULL + 2 * qt + h), phase, abort, lim)) return false;
+                    ptx::tc_fence_after();
+                    issue_o_half(p_tmem, vslot, d_tmem, acc, h);
+                }
+                return true;
             };
             bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort, lim) &&
                       ptx::mbar_wait(bar(C::B_KFULL + 0), 0, abort, lim);
@@ -288,12 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             for (int j = 0; ok && j < nkv; ++j) {
                 const int vs = j % C::VST;
                 if (!ptx::mbar_wait(bar(C::B_VFULL + vs), (j / C::VST) & 1, abort, lim) ||
-                    !ptx::mbar_wait(bar(C::B_PFULL + 0), j & 1, abort, lim)) {
+                    !issue_o(0, vs, j > 0, j & 1)) {
                     ok = false;
                     break;
                 }
-                ptx::tc_fence_after();
-                issue_o(tmem + C::COL_S0, vs, tmem + C::COL_O0, j > 0);
                 const bool more = j + 1 < nkv;
                 const int ks = (j + 1) % C::KST;
                 if (more) {
@@ -305,12 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     issue_s(qd0, ks, tmem + C::COL_S0);
                     ptx::mma_commit(bar(C::B_SFULL + 0));
                 }
-                if (!ptx::mbar_wait(bar(C::B_PFULL + 1), j & 1, abort, lim)) {
+                if (!issue_o(1, vs, j > 0, j & 1)) {
                     ok = false;
                     break;
                 }
-                ptx::tc_fence_after();
-                issue_o(tmem + C::COL_S1, vs, tmem + C::COL_O1, j > 0);
                 ptx::mma_commit(bar(C::B_VEMPTY + vs));
                 if (more) {
                     issue_s(qd1, ks, tmem + C::COL_S1);
@@ -340,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_base + (qt ? C::COL_S1 : C::COL_S0);
         const uint32_t o_col = qt ? C::COL_O1 : C::COL_O0;
-        const uint32_t sfull = bar(C::B_SFULL + qt), pfull = bar(C::B_PFULL + qt);
+        const uint32_t sfull = bar(C::B_SFULL + qt);
         // The two query tiles take turns on the MUFU unit (their exponential phases would
         // otherwise overlap and each would run at half rate).
         const uint32_t my_turn = bar(C::B_TURN + qt), other_turn = bar(C::B_TURN + (qt ^ 1));
@@ -356,123 +324,97 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             }
             ptx::tc_fence_after();
             const bool last = (j == nkv - 1);
-            uint32_t sv[kBN];
-            float sum = 0.f, alpha = 1.f;
-            if (!SKIPARSE_STALE_MAX || j == 0 || last) {
-                // The row max is taken over the whole tile before any exponential (the first
-                // tile sets the reference max; the ragged last tile has masked keys).
-                float sc[kBN];
+            // The row max is taken over the whole tile before any exponential (the first tile
+            // sets the reference max; the ragged last tile has masked keys).
+            float sc[kBN];
+            {
+                uint32_t sv[kBN];
 #pragma unroll
                 for (int g = 0; g < 4; ++g)
                     ptx::tmem_ld32(s_addr + 32 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * g]));
                 ptx::tmem_wait_ld();  // one wait for the whole 128-column row
 #pragma unroll
                 for (int e = 0; e < kBN; ++e) sc[e] = __uint_as_float(sv[e]);
-                if (last) {
-                    const int valid = n_c - j * kBN;
+            }
+            if (last) {
+                const int valid = n_c - j * kBN;
 #pragma unroll
-                    for (int e = 0; e < kBN; ++e)
-                        if (e >= valid) sc[e] = -INFINITY;
-                }
-                // row max with 3-input max instructions, four independent chains
-                float mx0 = ptx::max3f(sc[0], sc[1], sc[2]), mx1 = ptx::max3f(sc[3], sc[4], sc[5]);
-                float mx2 = ptx::max3f(sc[6], sc[7], sc[8]), mx3 = ptx::max3f(sc[9], sc[10], sc[11]);
+                for (int e = 0; e < kBN; ++e)
+                    if (e >= valid) sc[e] = -INFINITY;
+            }
+            // row max with 3-input max instructions, four independent chains
+            float mx0 = ptx::max3f(sc[0], sc[1], sc[2]), mx1 = ptx::max3f(sc[3], sc[4], sc[5]);
+            float mx2 = ptx::max3f(sc[6], sc[7], sc[8]), mx3 = ptx::max3f(sc[9], sc[10], sc[11]);
 #pragma unroll
-                for (int e = 12; e + 8 <= kBN; e += 8) {
-                    mx0 = ptx::max3f(mx0, sc[e], sc[e + 1]);
-                    mx1 = ptx::max3f(mx1, sc[e + 2], sc[e + 3]);
-                    mx2 = ptx::max3f(mx2, sc[e + 4], sc[e + 5]);
-                    mx3 = ptx::max3f(mx3, sc[e + 6], sc[e + 7]);
-                }
-                static_assert((kBN - 12) % 8 == 4, "tail of the max chains");
-                mx0 = ptx::max3f(mx0, sc[kBN - 4], sc[kBN - 3]);
-                mx1 = ptx::max3f(mx1, sc[kBN - 2], sc[kBN - 1]);
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-                if (j == 0 || mx > m_run + thresh) {
-                    alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
-                    m_run = mx;
-                }
-                if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
-                    ok = false;
-                    break;
-                }
-                const float neg = -m_run * sl2;
-                float sum0 = 0.f, sum1 = 0.f;
+            for (int e = 12; e + 8 <= kBN; e += 8) {
+                mx0 = ptx::max3f(mx0, sc[e], sc[e + 1]);
+                mx1 = ptx::max3f(mx1, sc[e + 2], sc[e + 3]);
+                mx2 = ptx::max3f(mx2, sc[e + 4], sc[e + 5]);
+                mx3 = ptx::max3f(mx3, sc[e + 6], sc[e + 7]);
+            }
+            static_assert((kBN - 12) % 8 == 4, "tail of the max chains");
+            mx0 = ptx::max3f(mx0, sc[kBN - 4], sc[kBN - 3]);
+            mx1 = ptx::max3f(mx1, sc[kBN - 2], sc[kBN - 1]);
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            float alpha = 1.f;
+            if (j == 0 || mx > m_run + thresh) {
+                alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
+                m_run = mx;
+            }
+            if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
+                ok = false;
+                break;
+            }
+            // P = 2^(S*scale*log2(e) - m), written as bf16 pairs over the first 64 columns of S.
+            // Each half of the key tile is released to the tensor core as soon as it is stored,
+            // so O += P V on the first half overlaps the exponentials of the second.
+            const float neg = -m_run * sl2;
+            float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint32_t pk[16];
+            for (int g = 0; g < 4; ++g) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float x0 = fmaf(sc[32 * g + 2 * e], sl2, neg);
-                        const float x1 = fmaf(sc[32 * g + 2 * e + 1], sl2, neg);
-                        float p0, p1;
-                        if (kEmuMask != 0u && !last && (kEmuMask & (1u << e))) {
-                            p0 = ptx::exp2_poly(x0);
-                            p1 = ptx::exp2_poly(x1);
-                        } else {
-                            p0 = ptx::ex2_approx(x0);
-                            p1 = ptx::ex2_approx(x1);
-                        }
-                        sum0 += p0;
-                        sum1 += p1;
-                        pk[e] = ptx::pack_bf16x2(p0, p1);
+                for (int e = 0; e < 16; ++e) {
+                    const float x0 = fmaf(sc[32 * g + 2 * e], sl2, neg);
+                    const float x1 = fmaf(sc[32 * g + 2 * e + 1], sl2, neg);
+                    float p0, p1;
+                    if (kEmuMask != 0u && !last && (kEmuMask & (1u << e))) {
+                        p0 = ptx::exp2_poly(x0);
+                        p1 = ptx::exp2_poly(x1);
+                    } else {
+                        p0 = ptx::ex2_approx(x0);
+                        p1 = ptx::ex2_approx(x1);
                     }
-                    ptx::tmem_st16(s_addr + 16 * g, pk);
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[e] = ptx::pack_bf16x2(p0, p1);
                 }
-                sum = sum0 + sum1;
-                if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
-            } else {
-                // Steady state: exponentials against the running max while the next 32-column
-                // chunk of S is loading; the tile's max is only checked afterwards.
-                if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
-                    ok = false;
-                    break;
-                }
-                const float neg = -m_run * sl2;
-                float mx = -INFINITY;
-                ptx::tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                ptx::tmem_wait_ld();
+                ptx::tmem_st16(s_addr + 16 * g, pk);
+                if (g == 1 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // Rare: a row max grew by more than 2^8. This warp rescales its rows of O_qt
+                    // before releasing the first half of P, i.e. before this tile's P*V
+                    // accumulates into O_qt; O_qt was completed by the previous P*V (the commit
+                    // behind this tile's S covers it). Half of the scores are consumed here,
+                    // which leaves room in registers.
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    if (g < 3)
-                        ptx::tmem_ld32(s_addr + 32 * (g + 1), *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * (g + 1)]));
-                    mx = fmaxf(mx, row_max<32>(&sv[32 * g]));
-                    sum += exp_chunk<true>(&sv[32 * g], sl2, neg, s_addr + 16 * g);
-                    if (g < 3) ptx::tmem_wait_ld();
-                }
-                if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
-                const bool grow = mx > m_run + thresh;
-                if (__any_sync(0xffffffffu, grow)) {
-                    // Rare: this tile raised a row max by more than 2^8. Redo its P against the
-                    // new max (S is still in registers) and rescale O below.
-                    if (grow) {
-                        alpha = ptx::ex2_approx((m_run - mx) * sl2);
-                        m_run = mx;
+                    for (int go = 0; go < D / 32; ++go) {
+                        uint32_t ov[32];
+                        const uint32_t o_addr = tmem + lane_base + o_col + 32 * go;
+                        ptx::tmem_ld32(o_addr, ov);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        ptx::tmem_st32(o_addr, ov);
                     }
-                    const float neg2 = -m_run * sl2;
-                    ptx::tmem_wait_st();  // the first pass's stores land before they are redone
-                    sum = 0.f;
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) sum += exp_chunk<false>(&sv[32 * g], sl2, neg2, s_addr + 16 * g);
+                }
+                if (g & 1) {
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(bar(C::B_PFULL + 2 * qt + (g >> 1)));
                 }
             }
-            l_run = l_run * alpha + sum;
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                // O_qt was completed by the previous P*V (the commit behind this tile's S covers it)
-#pragma unroll
-                for (int g = 0; g < D / 32; ++g) {
-                    uint32_t ov[32];
-                    const uint32_t o_addr = tmem + lane_base + o_col + 32 * g;
-                    ptx::tmem_ld32(o_addr, ov);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                    ptx::tmem_st32(o_addr, ov);
-                }
-            }
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(pfull);
+            if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
+            l_run = l_run * alpha + (sum0 + sum1);
         }
         if (ok && ptx::mbar_wait(bar(C::B_OFULL), 0, abort, lim)) {
             ptx::tc_fence_after();
