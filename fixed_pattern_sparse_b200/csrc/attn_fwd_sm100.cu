@@ -53,7 +53,13 @@ constexpr int kLaunchRegs = 168;       // 65536 / 384 rounded down to a multiple
 constexpr int kProdWarp0 = 8;
 constexpr int kNumProducers = 64;
 constexpr int kMmaWarp = 10;
-constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+constexpr float kRescaleLog2 = 8.0f;
+// P is released to the tensor core in this many parts of the key tile (2 or 4).
+#ifndef SKIPARSE_P_PARTS
+#define SKIPARSE_P_PARTS 2
+#endif
+constexpr int kPParts = SKIPARSE_P_PARTS;
+static_assert(kPParts == 2 || kPParts == 4, "P parts");  // rescale O only when the max grows by more than 2^8
 // Which of the 16 column pairs of every 32-column chunk take exp2 on the FMA pipe (polynomial)
 // instead of the MUFU unit. 0: none (fastest measured: MUFU is not this kernel's limiter).
 #ifndef SKIPARSE_EMU_MASK
@@ -85,8 +91,8 @@ struct Cfg : TileGeom<D> {
     static constexpr int B_VFULL = B_KEMPTY + KST;
     static constexpr int B_VEMPTY = B_VFULL + VST;
     static constexpr int B_SFULL = B_VEMPTY + VST;        // 2: one per query tile
-    static constexpr int B_PFULL = B_SFULL + 2;           // 4: (query tile, half of the key tile)
-    static constexpr int B_TURN = B_PFULL + 4;            // 2: MUFU turn of query tile 0 / 1
+    static constexpr int B_PFULL = B_SFULL + 2;           // 2 x kPParts: (query tile, part of the key tile)
+    static constexpr int B_TURN = B_PFULL + 2 * kPParts;  // 2: MUFU turn of query tile 0 / 1
     static constexpr int B_OFULL = B_TURN + 2;
     static constexpr int B_DRAIN = B_OFULL + 1;
     static constexpr int NBARS = B_DRAIN + 1;
@@ -141,8 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
-            ptx::mbar_init(bar(C::B_PFULL + 2 * i), kBM);
-            ptx::mbar_init(bar(C::B_PFULL + 2 * i + 1), kBM);
+            for (int h = 0; h < kPParts; ++h) ptx::mbar_init(bar(C::B_PFULL + kPParts * i + h), kBM);
             ptx::mbar_init(bar(C::B_TURN + i), kBM);
         }
         ptx::mbar_init(bar(C::B_OFULL), 1);
@@ -226,13 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     ptx::mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
-            // O += P V over one half of the key tile (keys [64h, 64h+64)), as soon as the softmax
-            // has released that half of P
+            // O += P V over one part of the key tile (keys [h, h+1) * kBN / kPParts), as soon as
+            // the softmax has released that part of P
             auto issue_o_half = [&](uint32_t p_tmem, int vslot, uint32_t d_tmem, bool acc, int h) {
                 const uint64_t vd = vd0 + ((vslot * C::TILE_BYTES) >> 4);
+                constexpr int KPP = kBN / 16 / kPParts;  // K-steps per part
 #pragma unroll
-                for (int k4 = 0; k4 < kBN / 32; ++k4) {
-                    const int kk = h * (kBN / 32) + k4;
+                for (int k4 = 0; k4 < KPP; ++k4) {
+                    const int kk = h * KPP + k4;
                     ptx::mma_ts(d_tmem, p_tmem + kk * 8, vd + ((kk * 16 * C::SW) >> 4), idesc_o,
                                 (acc || kk > 0) ? 1u : 0u);
                 }
@@ -240,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             auto issue_o = [&](int qt, int vslot, bool acc, int phase) -> bool {
                 const uint32_t p_tmem = tmem + (qt ? C::COL_S1 : C::COL_S0);
                 const uint32_t d_tmem = tmem + (qt ? C::COL_O1 : C::COL_O0);
-                for (int h = 0; h < 2; ++h) {
-                    if (!ptx::mbar_wait(bar(C::B_PFULL + 2 * qt + h), phase, abort, lim)) return false;
+                for (int h = 0; h < kPParts; ++h) {
+                    if (!ptx::mbar_wait(bar(C::B_PFULL + kPParts * qt + h), phase, abort, lim)) return false;
                     ptx::tc_fence_after();
                     issue_o_half(p_tmem, vslot, d_tmem, acc, h);
                 }
@@ -390,27 +396,27 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     pk[e] = ptx::pack_bf16x2(p0, p1);
                 }
                 ptx::tmem_st16(s_addr + 16 * g, pk);
-                if (g == 1 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (g == (kPParts == 4 ? 0 : 1) && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     // Rare: a row max grew by more than 2^8. This warp rescales its rows of O_qt
                     // before releasing the first half of P, i.e. before this tile's P*V
                     // accumulates into O_qt; O_qt was completed by the previous P*V (the commit
                     // behind this tile's S covers it). Half of the scores are consumed here,
                     // which leaves room in registers.
 #pragma unroll
-                    for (int go = 0; go < D / 32; ++go) {
-                        uint32_t ov[32];
-                        const uint32_t o_addr = tmem + lane_base + o_col + 32 * go;
-                        ptx::tmem_ld32(o_addr, ov);
+                    for (int go = 0; go < D / 16; ++go) {
+                        uint32_t ov[16];
+                        const uint32_t o_addr = tmem + lane_base + o_col + 16 * go;
+                        ptx::tmem_ld16(o_addr, ov);
                         ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        ptx::tmem_st32(o_addr, ov);
+                        for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        ptx::tmem_st16(o_addr, ov);
                     }
                 }
-                if (g & 1) {
+                if (kPParts == 4 || (g & 1)) {
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
-                    ptx::mbar_arrive(bar(C::B_PFULL + 2 * qt + (g >> 1)));
+                    ptx::mbar_arrive(bar(C::B_PFULL + kPParts * qt + (kPParts == 4 ? g : g >> 1)));
                 }
             }
             if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
