@@ -13,6 +13,8 @@
 //      in TMEM (TMEM: S^T, dP^T, dV, dK = 512 columns);
 //   3. query-major kernel (KV = false): a CTA keeps one 128-query tile (Q, dO, L, D) and streams
 //      the class's key tiles (K, V): S, dP into TMEM, dS, then dQ += dS K in TMEM.
+// The MMA issuer runs one streamed tile ahead: the next tile's S (and dP) are computed while
+// the softmax warps work on the current tile.
 // No atomics: every gradient row is produced by exactly one CTA, so results are deterministic.
 // Warp roles (11 warps): two softmax warpgroups (each owns 64 of the 128 streamed columns of
 // every TMEM row), two producer warps (16-byte cp.async gathers of class rows into the UMMA
@@ -48,7 +50,7 @@ struct BwdCfg : TileGeom<D> {
     static constexpr int VEC_BYTES = 2 * 2 * kTileRows * 4;
     static constexpr int OFF_BAR = OFF_VEC + VEC_BYTES;
     static constexpr int B_STAT = 0, B_FULL = 1, B_EMPTY = 3, B_X1 = 5, B_X2 = 6, B_P = 7, B_DS = 8,
-                         B_ACC = 9, B_DRAIN = 10, NBARS = 11;
+                         B_ACC = 9, B_DRAIN = 10, B_X1FREE = 11, NBARS = 12;
     static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
     static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
     static constexpr int SMEM_USED = OFF_ABORT + 4;
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         ptx::mbar_init(bar(C::B_X2), 1);
         ptx::mbar_init(bar(C::B_P), kBwdSoftmax);
         ptx::mbar_init(bar(C::B_DS), kBwdSoftmax);
+        ptx::mbar_init(bar(C::B_X1FREE), kBwdSoftmax);
         ptx::mbar_init(bar(C::B_ACC), 1);
         ptx::mbar_init(bar(C::B_DRAIN), 1);
         *abort = 0;
@@ -146,8 +149,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             load_vec(sbase + C::OFF_VEC, p.lse, ta, pw, lane);
             load_vec(sbase + C::OFF_VEC + 4 * kTileRows, p.delta, ta, pw, lane);
         }
-        cp_async_commit();
-        uint32_t prev_bar = bar(C::B_STAT);
+        cp_async_arrive_noinc(bar(C::B_STAT));
         bool ok = true;
         for (int j = 0; j < nstream; ++j) {
             const int s = j & 1;
@@ -169,19 +171,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 load_vec(v, p.lse, tr, pw, lane);
                 load_vec(v + 4 * kTileRows, p.delta, tr, pw, lane);
             }
-            cp_async_commit();
-            cp_async_wait<1>();
-            fence_proxy_async();
-            ptx::mbar_arrive(prev_bar);
-            prev_bar = bar(C::B_FULL + s);
+            cp_async_arrive_noinc(bar(C::B_FULL + s));  // completes when this tile has landed
         }
-        cp_async_wait<0>();
-        if (ok) {
-            fence_proxy_async();
-            ptx::mbar_arrive(prev_bar);
-        } else {
-            record_abort(abort, p.status);
-        }
+        cp_async_commit();
+        cp_async_wait<0>();  // no copy of this thread outlives it
+        if (!ok) record_abort(abort, p.status);
     } else if (warp == kBwdMma) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -204,22 +198,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                     ptx::mma_ts(d_tmem, tmem + a_col + half_packed_col(kk), bm + ((kk * 16 * C::SW) >> 4),
                                 idesc_acc, (acc || kk > 0) ? 1u : 0u);
             };
+            // Issue order per streamed tile j, so that the softmax of one tile overlaps the tensor
+            // core's work on its neighbours (every MMA below reuses a TMEM region only after the
+            // MMA that last read it, in issue order):
+            //   key-major  : dV(j) [P(j)], X1(j+1), dK(j) [dS(j)], X2(j+1)
+            //   query-major: X1(j+1) [S(j) read by the softmax], dQ(j) [dS(j)], X2(j+1)
+            auto issue_x1 = [&](int j) -> bool {   // S (or S^T) of streamed tile j
+                const int s = j & 1;
+                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) return false;
+                fence_proxy_async();  // the cp.async data, observed through the barrier, for the MMA
+                ptx::tc_fence_after();
+                x_mma(a1, bk0 + ((2 * s * C::TILE_BYTES) >> 4), tmem + C::COL_X1);
+                ptx::mma_commit(bar(C::B_X1));
+                return true;
+            };
+            auto issue_x2 = [&](int j) {           // dP (or dP^T); tile j's slot already waited
+                const int s = j & 1;
+                x_mma(a2, bk0 + (((2 * s + 1) * C::TILE_BYTES) >> 4), tmem + C::COL_X2);
+                ptx::mma_commit(bar(C::B_X2));
+            };
             bool ok = ptx::mbar_wait(bar(C::B_STAT), 0, abort, lim);
+            fence_proxy_async();
+            ok = ok && issue_x1(0);
+            if (ok) issue_x2(0);
             for (int j = 0; ok && j < nstream; ++j) {
                 const int s = j & 1;
-                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const uint64_t b1k = bk0 + ((2 * s * C::TILE_BYTES) >> 4);
-                const uint64_t b2k = bk0 + (((2 * s + 1) * C::TILE_BYTES) >> 4);
+                const bool more = j + 1 < nstream;
                 const uint64_t b1m = bm0 + ((2 * s * C::TILE_BYTES) >> 4);
                 const uint64_t b2m = bm0 + (((2 * s + 1) * C::TILE_BYTES) >> 4);
-                x_mma(a1, b1k, tmem + C::COL_X1);
-                ptx::mma_commit(bar(C::B_X1));
-                x_mma(a2, b2k, tmem + C::COL_X2);
-                ptx::mma_commit(bar(C::B_X2));
                 if (KV) {
                     if (!ptx::mbar_wait(bar(C::B_P), j & 1, abort, lim)) {
                         ok = false;
@@ -227,6 +233,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                     }
                     ptx::tc_fence_after();
                     acc_mma(C::COL_X1, b2m, tmem + C::COL_ACC1, j > 0);   // dV += P^T dO
+                } else if (!ptx::mbar_wait(bar(C::B_X1FREE), j & 1, abort, lim)) {
+                    ok = false;
+                    break;
+                }
+                if (more && !issue_x1(j + 1)) {
+                    ok = false;
+                    break;
                 }
                 if (!ptx::mbar_wait(bar(C::B_DS), j & 1, abort, lim)) {
                     ok = false;
@@ -236,6 +249,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 // key-major: dK += dS^T Q ; query-major: dQ += dS K
                 acc_mma(C::COL_X2, b1m, tmem + (KV ? C::COL_ACC2 : C::COL_ACC1), j > 0);
                 ptx::mma_commit(bar(C::B_EMPTY + s));
+                if (more) issue_x2(j + 1);
             }
             if (ok) {
                 ptx::mma_commit(bar(C::B_ACC));
@@ -282,6 +296,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 ptx::tmem_ld32(x1, *reinterpret_cast<uint32_t(*)[32]>(&xv[0]));
                 ptx::tmem_ld32(x1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&xv[32]));
                 ptx::tmem_wait_ld();
+                if (!KV) {  // S is in registers: the tensor core may compute the next tile's S
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(bar(C::B_X1FREE));
+                }
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     const float l2 = KV ? col_l[e] * kLog2e : row_l2;
