@@ -170,15 +170,14 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
 #endif
       if (warp == kProdWarp0 || warp == kProdWarp0 + 1) {
         // ------------------------------------------------------------------ producers
-        // Load order Q, K0, V0, K1, V1, ... Each load is one cp.async group; a load's full
-        // barrier is signalled (after this thread's copies completed and a proxy fence) once
-        // the next load has been issued, so two loads are in flight per thread.
+        // Load order Q, K0, V0, K1, V1, ... Every thread arrives on a load's full barrier with
+        // cp.async.mbarrier.arrive.noinc right after issuing its copies; the arrival fires when
+        // they have landed, so a tile is released as soon as it is in shared memory.
         const int pw = warp - kProdWarp0;
         const int fault_skip = (p.fault == 1 && pw == 0 && lane == 0);
         load_tile<D>(sbase + C::OFF_Q, p.q, rows, q_first, n_c, pw, lane);
         load_tile<D>(sbase + C::OFF_Q + C::TILE_BYTES, p.q, rows, q_first + kBM, n_c, pw, lane);
-        cp_async_commit();
-        uint32_t prev_bar = bar(C::B_Q);
+        cp_async_arrive_noinc(bar(C::B_Q));
         bool ok = true;
         TileRows kv{0, 0};  // token rows of key step j, shared by its K and V tiles
         for (int L = 0; L < 2 * nkv; ++L) {
@@ -199,19 +198,12 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             }
             const uint32_t dst = sbase + (is_v ? C::OFF_V : C::OFF_K) + s * C::TILE_BYTES;
             load_tile_rows<D>(dst, is_v ? p.v : p.k, kv, pw, lane);
-            cp_async_commit();
-            cp_async_wait<1>();   // the previous load has landed
-            fence_proxy_async();  // make it visible to the tensor core (async proxy)
-            if (!(fault_skip && L == 1)) ptx::mbar_arrive(prev_bar);
-            prev_bar = bar((is_v ? C::B_VFULL : C::B_KFULL) + s);
+            // test hook: one thread never signals the first K tile
+            if (!(fault_skip && L == 0)) cp_async_arrive_noinc(bar((is_v ? C::B_VFULL : C::B_KFULL) + s));
         }
-        cp_async_wait<0>();
-        if (ok) {
-            fence_proxy_async();
-            ptx::mbar_arrive(prev_bar);
-        } else {
-            record_abort(abort, p.status);
-        }
+        cp_async_commit();
+        cp_async_wait<0>();  // no copy of this thread outlives it
+        if (!ok) record_abort(abort, p.status);
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -256,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             bool ok = ptx::mbar_wait(bar(C::B_Q), 0, abort, lim) &&
                       ptx::mbar_wait(bar(C::B_KFULL + 0), 0, abort, lim);
             if (ok) {
+                fence_proxy_async();  // cp.async data observed through the barriers, for the MMA
                 ptx::tc_fence_after();
                 issue_s(qd0, 0, tmem + C::COL_S0);
                 ptx::mma_commit(bar(C::B_SFULL + 0));
@@ -265,8 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const int vs = j % C::VST;
-                if (!ptx::mbar_wait(bar(C::B_VFULL + vs), (j / C::VST) & 1, abort, lim) ||
-                    !issue_o(0, vs, j > 0, j & 1)) {
+                const bool v_ok = ptx::mbar_wait(bar(C::B_VFULL + vs), (j / C::VST) & 1, abort, lim);
+                if (v_ok) fence_proxy_async();
+                if (!v_ok || !issue_o(0, vs, j > 0, j & 1)) {
                     ok = false;
                     break;
                 }
@@ -277,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                         ok = false;
                         break;
                     }
+                    fence_proxy_async();
                     ptx::tc_fence_after();
                     issue_s(qd0, ks, tmem + C::COL_S0);
                     ptx::mma_commit(bar(C::B_SFULL + 0));
