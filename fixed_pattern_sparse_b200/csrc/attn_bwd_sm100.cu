@@ -16,9 +16,10 @@
 // The MMA issuer runs one streamed tile ahead: the next tile's S (and dP) are computed while
 // the softmax warps work on the current tile.
 // No atomics: every gradient row is produced by exactly one CTA, so results are deterministic.
-// Warp roles (11 warps): two softmax warpgroups (each owns 64 of the 128 streamed columns of
-// every TMEM row), two producer warps (16-byte cp.async gathers of class rows into the UMMA
-// swizzled layout, 4-byte cp.async for L and D), one MMA warp (tcgen05.mma, one thread).
+// Warp roles (13 warps): two softmax warpgroups (each owns 64 of the 128 streamed columns of
+// every TMEM row), four producer warps (16-byte cp.async gathers of class rows into the UMMA
+// swizzled layout, one pair per streamed tensor, 4-byte cp.async for L and D), one MMA warp
+// (tcgen05.mma, one thread).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -27,10 +28,12 @@
 namespace skiparse {
 namespace {
 
-constexpr int kBwdThreads = 352;
+// 13 warps: softmax 0-7, producers 8-11 (warps 8-9 copy the first streamed tensor and the
+// statistics, warps 10-11 the second, each pair splitting a tile's rows), MMA issuer 12.
+constexpr int kBwdThreads = 416;
 constexpr int kBwdProd0 = 8;
-constexpr int kBwdProducers = 64;
-constexpr int kBwdMma = 10;
+constexpr int kBwdProducers = 128;
+constexpr int kBwdMma = 12;
 constexpr int kBwdSoftmax = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -49,8 +52,9 @@ struct BwdCfg : TileGeom<D> {
     static constexpr int OFF_VEC = OFF_B + 4 * TILE_BYTES;    // [slot or stationary][L,D][128] fp32
     static constexpr int VEC_BYTES = 2 * 2 * kTileRows * 4;
     static constexpr int OFF_BAR = OFF_VEC + VEC_BYTES;
-    static constexpr int B_STAT = 0, B_FULL = 1, B_EMPTY = 3, B_X1 = 5, B_X2 = 6, B_P = 7, B_DS = 8,
-                         B_ACC = 9, B_DRAIN = 10, B_X1FREE = 11, NBARS = 12;
+    // B_FULL / B_EMPTY: [tensor (0: B1, 1: B2)][slot], index B_FULL + 2 * tensor + slot
+    static constexpr int B_STAT = 0, B_FULL = 1, B_EMPTY = 5, B_X1 = 9, B_X2 = 10, B_P = 11, B_DS = 12,
+                         B_ACC = 13, B_DRAIN = 14, B_X1FREE = 15, NBARS = 16;
     static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
     static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
     static constexpr int SMEM_USED = OFF_ABORT + 4;
@@ -110,9 +114,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(C::B_STAT), kBwdProducers);
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(bar(C::B_FULL + s), kBwdProducers);
-            ptx::mbar_init(bar(C::B_EMPTY + s), 1);
+        for (int i = 0; i < 4; ++i) {
+            ptx::mbar_init(bar(C::B_FULL + i), kBwdProducers / 2);  // one producer pair per tensor
+            ptx::mbar_init(bar(C::B_EMPTY + i), 1);
         }
         ptx::mbar_init(bar(C::B_X1), 1);
         ptx::mbar_init(bar(C::B_X2), 1);
@@ -139,13 +143,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
     const uint16_t* g_b1 = KV ? p.q : p.k;
     const uint16_t* g_b2 = KV ? p.dout : p.v;
 
-    if (warp == kBwdProd0 || warp == kBwdProd0 + 1) {
+    if (warp >= kBwdProd0 && warp < kBwdProd0 + 4) {
         // ------------------------------------------------------------------ producers
-        const int pw = warp - kBwdProd0;
+        // Pair 0 (warps 8-9) copies the first tensor of every tile (and the L/D statistics),
+        // pair 1 (warps 10-11) the second; within a pair, warp pw copies rows [64pw, 64pw+64).
+        const int pair = (warp - kBwdProd0) >> 1;
+        const int pw = (warp - kBwdProd0) & 1;
         const TileRows ta = tile_rows(rows, first, n_c, pw, lane);
-        load_tile_rows<D>(sbase + C::OFF_A1, g_a1, ta, pw, lane);
-        load_tile_rows<D>(sbase + C::OFF_A2, g_a2, ta, pw, lane);
-        if (!KV) {  // the stationary queries' L and D
+        load_tile_rows<D>(sbase + (pair ? C::OFF_A2 : C::OFF_A1), pair ? g_a2 : g_a1, ta, pw, lane);
+        if (!KV && pair == 0) {  // the stationary queries' L and D
             load_vec(sbase + C::OFF_VEC, p.lse, ta, pw, lane);
             load_vec(sbase + C::OFF_VEC + 4 * kTileRows, p.delta, ta, pw, lane);
         }
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             const int s = j & 1;
             if (j >= 2) {
                 int w_ok = 1;
-                if (lane == 0) w_ok = ptx::mbar_wait(bar(C::B_EMPTY + s), ((j >> 1) - 1) & 1, abort, lim);
+                if (lane == 0) w_ok = ptx::mbar_wait(bar(C::B_EMPTY + 2 * pair + s), ((j >> 1) - 1) & 1, abort, lim);
                 w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                 if (!w_ok) {
                     ok = false;
@@ -164,14 +170,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             }
             const uint32_t slot = sbase + C::OFF_B + 2 * s * C::TILE_BYTES;
             const TileRows tr = tile_rows(rows, j * kTileRows, n_c, pw, lane);
-            load_tile_rows<D>(slot, g_b1, tr, pw, lane);
-            load_tile_rows<D>(slot + C::TILE_BYTES, g_b2, tr, pw, lane);
-            if (KV) {  // the streamed queries' L and D
+            load_tile_rows<D>(slot + (pair ? C::TILE_BYTES : 0), pair ? g_b2 : g_b1, tr, pw, lane);
+            if (KV && pair == 0) {  // the streamed queries' L and D
                 const uint32_t v = sbase + C::OFF_VEC + s * 2 * 4 * kTileRows;
                 load_vec(v, p.lse, tr, pw, lane);
                 load_vec(v + 4 * kTileRows, p.delta, tr, pw, lane);
             }
-            cp_async_arrive_noinc(bar(C::B_FULL + s));  // completes when this tile has landed
+            cp_async_arrive_noinc(bar(C::B_FULL + 2 * pair + s));  // completes when this tile has landed
         }
         cp_async_commit();
         cp_async_wait<0>();  // no copy of this thread outlives it
@@ -205,22 +210,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             //   query-major: X1(j+1) [S(j) read by the softmax], dQ(j) [dS(j)], X2(j+1)
             auto issue_x1 = [&](int j) -> bool {   // S (or S^T) of streamed tile j
                 const int s = j & 1;
-                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) return false;
+                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) return false;  // B1
                 fence_proxy_async();  // the cp.async data, observed through the barrier, for the MMA
                 ptx::tc_fence_after();
                 x_mma(a1, bk0 + ((2 * s * C::TILE_BYTES) >> 4), tmem + C::COL_X1);
                 ptx::mma_commit(bar(C::B_X1));
                 return true;
             };
-            auto issue_x2 = [&](int j) {           // dP (or dP^T); tile j's slot already waited
+            auto issue_x2 = [&](int j) -> bool {   // dP (or dP^T) of streamed tile j
                 const int s = j & 1;
+                if (!ptx::mbar_wait(bar(C::B_FULL + 2 + s), (j >> 1) & 1, abort, lim)) return false;  // B2
+                fence_proxy_async();
+                ptx::tc_fence_after();
                 x_mma(a2, bk0 + (((2 * s + 1) * C::TILE_BYTES) >> 4), tmem + C::COL_X2);
                 ptx::mma_commit(bar(C::B_X2));
+                if (!KV) ptx::mma_commit(bar(C::B_EMPTY + 2 + s));  // V_j: dP was its last reader
+                return true;
             };
             bool ok = ptx::mbar_wait(bar(C::B_STAT), 0, abort, lim);
             fence_proxy_async();
-            ok = ok && issue_x1(0);
-            if (ok) issue_x2(0);
+            ok = ok && issue_x1(0) && issue_x2(0);
             for (int j = 0; ok && j < nstream; ++j) {
                 const int s = j & 1;
                 const bool more = j + 1 < nstream;
@@ -233,6 +242,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                     }
                     ptx::tc_fence_after();
                     acc_mma(C::COL_X1, b2m, tmem + C::COL_ACC1, j > 0);   // dV += P^T dO
+                    ptx::mma_commit(bar(C::B_EMPTY + 2 + s));             // dO_j: dV was its last reader
                 } else if (!ptx::mbar_wait(bar(C::B_X1FREE), j & 1, abort, lim)) {
                     ok = false;
                     break;
@@ -248,8 +258,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 ptx::tc_fence_after();
                 // key-major: dK += dS^T Q ; query-major: dQ += dS K
                 acc_mma(C::COL_X2, b1m, tmem + (KV ? C::COL_ACC2 : C::COL_ACC1), j > 0);
-                ptx::mma_commit(bar(C::B_EMPTY + s));
-                if (more) issue_x2(j + 1);
+                ptx::mma_commit(bar(C::B_EMPTY + s));  // B1 of tile j: dK / dQ was its last reader
+                if (more && !issue_x2(j + 1)) {
+                    ok = false;
+                    break;
+                }
             }
             if (ok) {
                 ptx::mma_commit(bar(C::B_ACC));
