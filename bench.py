@@ -51,6 +51,9 @@ KNOWN_TRAFFIC = {
     "2a906497c379c4ad": 2.955e9,
     # the per-axis class-count kernel: 480p capture 302.5 + 80.1 MB per launch, x 7.692
     "726002548e064429": 2.943e9,
+    # measured directly on the 720p launch (one-pass dram__bytes metrics): 2.33 GB read +
+    # 0.756 GB written = q, k, v read once and out written once
+    "5d623923e1bf3aa7": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
