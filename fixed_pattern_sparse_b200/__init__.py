@@ -21,7 +21,8 @@ __all__ = ["TOKEN_WISE", "GROUP_WISE", "SkiparseError", "skiparse2d_attn_fwd", "
            "get_device_status", "attn_fwd_from_host", "HostStaging", "attn_flops", "STATUS",
            "skiparse2d_attn_fwd_lse", "skiparse2d_attn_bwd", "SkiparseAttention", "skiparse_attention",
            "skiparse1d_attn_fwd", "skiparse1d_attn_fwd_lse", "skiparse1d_attn_bwd", "skiparse1d_rearrange",
-           "skiparse1d_unrearrange", "skiparse1d_switch_mode", "padded_length_1d"]
+           "skiparse1d_unrearrange", "skiparse1d_switch_mode", "padded_length_1d", "attn_fwd_host",
+           "host_workspace_bytes"]
 
 
 def _stream_ptr(stream) -> int:
@@ -299,6 +300,39 @@ def skiparse1d_switch_mode(y: torch.Tensor, shape, P: int, src_mode: int, out: t
 def get_device_status(stream=None) -> int:
     """Synchronizes the stream; returns and clears the device error word (0 = OK)."""
     return lib().skiparse_get_device_status(_stream_ptr(stream))
+
+
+def host_workspace_bytes(shape, heads_per_group: int) -> int:
+    B, T, H, W, heads, d = shape
+    return lib().skiparse_attn_fwd_host_workspace_bytes(B, T, H, W, heads, d, heads_per_group)
+
+
+def attn_fwd_host(q_host: torch.Tensor, k_host: torch.Tensor, v_host: torch.Tensor, P: int, mode: int,
+                  out_host: torch.Tensor, heads_per_group: int = 8, workspace: torch.Tensor | None = None,
+                  dims: int = 2, stream=None) -> torch.Tensor:
+    """The forward with HOST buffers (skiparse2d_attn_fwd_host / skiparse1d_attn_fwd_host): q, k, v
+    and out are CPU bf16 tensors of one (B,T,H,W,heads,d) shape (pinned memory lets the library
+    overlap its copies with the kernel); `workspace` is a CUDA uint8 tensor of at least
+    host_workspace_bytes(shape, heads_per_group) bytes (allocated here when not given).
+    Asynchronous on `stream`: synchronize it before reading out_host."""
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host), ("out_host", out_host)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor")
+        if t.shape != q_host.shape or t.dim() != 6:
+            raise ValueError("q, k, v, out must share one (B,T,H,W,heads,d) shape")
+    B, T, H, W, heads, d = q_host.shape
+    need = host_workspace_bytes(q_host.shape, heads_per_group)
+    if need < 0:
+        raise ValueError("invalid shape or heads_per_group")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or workspace.numel() < need:
+        raise ValueError(f"workspace must be a CUDA uint8 tensor of at least {need} bytes")
+    name = "skiparse2d_attn_fwd_host" if dims == 2 else "skiparse1d_attn_fwd_host"
+    check(getattr(lib(), name)(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), out_host.data_ptr(),
+                               B, T, H, W, heads, d, P, mode, heads_per_group, workspace.data_ptr(),
+                               workspace.numel(), _stream_ptr(stream)), name)
+    return out_host
 
 
 class HostStaging:

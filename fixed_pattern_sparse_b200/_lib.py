@@ -43,6 +43,9 @@ SIGNATURES = {
     "skiparse1d_subseq_len": (_LL, [_I] * 4),
     "skiparse1d_class_len": (_LL, [_I] * 6),
     "skiparse1d_rearranged_numel": (_LL, [_I] * 7),
+    "skiparse2d_attn_fwd_host": (_I, [_VP] * 4 + [_I] * 9 + [_VP, ctypes.c_size_t, _VP]),
+    "skiparse1d_attn_fwd_host": (_I, [_VP] * 4 + [_I] * 9 + [_VP, ctypes.c_size_t, _VP]),
+    "skiparse_attn_fwd_host_workspace_bytes": (_LL, [_I] * 7),
 }
 
 STATUS = {0: "SKIPARSE_OK", 1: "SKIPARSE_ERR_INVALID_ARG", 2: "SKIPARSE_ERR_UNSUPPORTED",

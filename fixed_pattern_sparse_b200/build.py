@@ -17,7 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libskiparse.so")
-SOURCES = ["skiparse_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "rearrange.cu", "no_alloc.cu"]
+SOURCES = ["skiparse_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "rearrange.cu", "no_alloc.cu",
+           "host_pipeline.cu"]
 HEADERS = ["ptx_sm100.cuh", "skiparse_internal.cuh", "attn_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

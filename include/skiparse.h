@@ -32,6 +32,8 @@
 #ifndef SKIPARSE_H
 #define SKIPARSE_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -169,6 +171,37 @@ SKIPARSE_API long long skiparse_subseq_len(int T, int H, int W, int P);
 SKIPARSE_API long long skiparse_class_len(int T, int H, int W, int P, int mode, int ci, int cj);
 
 /*
+ * The forward called with HOST buffers: q, k, v are read from host memory and out is written to
+ * host memory within the call (the same layouts and results as skiparse2d_attn_fwd). Heads are
+ * independent in the method (every (class, head) subsequence attends on its own), so the call is
+ * cut into groups of `heads_per_group` heads: a group's rows are copied in (one pitched copy per
+ * tensor), the fused kernel runs on it, and its output is copied out, with the copies of one
+ * group overlapping the kernel of another (library-owned streams, two workspace buffer sets).
+ *   q, k, v, out    : host pointers, (B, T, H, W, heads, d) bf16. Pinned (page-locked) memory
+ *                     lets the copies overlap; pageable memory gives the same results, slower.
+ *                     out must not overlap q, k or v.
+ *   heads_per_group : 1 <= heads_per_group <= heads; the last group may be smaller.
+ *   workspace       : device memory owned by the caller, 256-byte aligned, of at least
+ *                     skiparse_attn_fwd_host_workspace_bytes(B, T, H, W, heads, d,
+ *                     heads_per_group) bytes; it must not be used by anything else until the
+ *                     call has completed on `stream`.
+ * Asynchronous on `stream` like every entry point: the call starts after earlier work on
+ * `stream` and later work on `stream` (e.g. a synchronize) sees out written. Calls on one
+ * device are enqueued under a lock and run on the same internal streams, one after another.
+ * Errors: as skiparse2d_attn_fwd, plus SKIPARSE_ERR_INVALID_ARG for a bad group size or a small
+ * workspace, SKIPARSE_ERR_MISALIGNED for an unaligned workspace.
+ */
+SKIPARSE_API int skiparse2d_attn_fwd_host(const void* q, const void* k, const void* v, void* out,
+                                          int B, int T, int H, int W, int heads, int d, int P,
+                                          int mode, int heads_per_group, void* workspace,
+                                          size_t workspace_bytes, skiparse_stream_t stream);
+
+/* Device workspace bytes for skiparse2d_attn_fwd_host / skiparse1d_attn_fwd_host: two sets of
+ * four (B, T, H, W, heads_per_group, d) bf16 buffers; -1 on invalid arguments. */
+SKIPARSE_API long long skiparse_attn_fwd_host_workspace_bytes(int B, int T, int H, int W, int heads,
+                                                              int d, int heads_per_group);
+
+/*
  * ---- Skiparse-1D ------------------------------------------------------------------------
  * The 1D skip pattern on the flattened sequence, the variant that the summary page's sections
  * 技术新颖性 (novelty) and 实验结果 (results) compare Skiparse-2D with; the pages give no formula
@@ -190,6 +223,10 @@ SKIPARSE_API int skiparse1d_attn_fwd(const void* q, const void* k, const void* v
 SKIPARSE_API int skiparse1d_attn_fwd_lse(const void* q, const void* k, const void* v, void* out,
                                          float* lse, int B, int T, int H, int W, int heads, int d,
                                          int P, int mode, skiparse_stream_t stream);
+SKIPARSE_API int skiparse1d_attn_fwd_host(const void* q, const void* k, const void* v, void* out,
+                                          int B, int T, int H, int W, int heads, int d, int P,
+                                          int mode, int heads_per_group, void* workspace,
+                                          size_t workspace_bytes, skiparse_stream_t stream);
 SKIPARSE_API int skiparse1d_attn_bwd(const void* q, const void* k, const void* v, const void* out,
                                      const void* dout, const float* lse, void* dq, void* dk,
                                      void* dv, float* delta, int B, int T, int H, int W, int heads,

@@ -168,3 +168,20 @@ def test_product_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower().replace("oracles", ""), f
+
+
+def test_host_entry_rejects_bad_arguments_synchronously(L):
+    """The host-buffer forward validates everything before it creates streams or enqueues."""
+    need = L.skiparse_attn_fwd_host_workspace_bytes(1, 2, 8, 8, 4, 32, 2)
+    assert need > 0
+    assert L.skiparse_attn_fwd_host_workspace_bytes(1, 2, 8, 8, 4, 32, 5) == -1   # group > heads
+    big = 1 << 40
+    args = (FAKE, FAKE + big, FAKE + 2 * big, FAKE + 3 * big, 1, 2, 8, 8, 4, 32, 2, 0)
+    assert L.skiparse2d_attn_fwd_host(*args, 2, FAKE + 4 * big, need - 1, None) == 1     # workspace small
+    assert L.skiparse2d_attn_fwd_host(*args, 0, FAKE + 4 * big, need, None) == 1         # group 0
+    assert L.skiparse2d_attn_fwd_host(*args, 2, FAKE + 4 * big + 16, need, None) == 3    # misaligned
+    assert L.skiparse2d_attn_fwd_host(*args[:10], 2, 7, 2, FAKE + 4 * big, need, None) == 1  # bad mode
+    assert L.skiparse2d_attn_fwd_host(*args[:9], 48, 2, 0, 2, FAKE + 4 * big, 1 << 40, None) == 2  # d = 48
+    over = (FAKE, FAKE + big, FAKE + 2 * big, FAKE + 64, 1, 2, 8, 8, 4, 32, 2, 0)       # out overlaps q
+    assert L.skiparse2d_attn_fwd_host(*over, 2, FAKE + 4 * big, need, None) == 1
+    assert L.skiparse1d_attn_fwd_host(*args, 2, FAKE + 4 * big, need - 1, None) == 1
