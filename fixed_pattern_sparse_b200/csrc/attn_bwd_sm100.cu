@@ -313,11 +313,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(bar(C::B_X1FREE));
                 }
+                // key-major: each column's L, four at a time (the same 64 values for every row)
+                float lcol[64];
+                if (KV) {
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const float l2 = KV ? col_l[e] * kLog2e : row_l2;
-                    const float pe = ptx::ex2_approx(fmaf(__uint_as_float(xv[e]), sl2, -l2));
-                    pr[e] = (64 * h + e < valid) ? pe : 0.f;   // fake (clamped) streamed rows: 0
+                    for (int e4 = 0; e4 < 16; ++e4) {
+                        const float4 l4 = reinterpret_cast<const float4*>(col_l)[e4];
+                        lcol[4 * e4] = l4.x * kLog2e;
+                        lcol[4 * e4 + 1] = l4.y * kLog2e;
+                        lcol[4 * e4 + 2] = l4.z * kLog2e;
+                        lcol[4 * e4 + 3] = l4.w * kLog2e;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    pr[e] = ptx::ex2_approx(fmaf(__uint_as_float(xv[e]), sl2, -(KV ? lcol[e] : row_l2)));
+                if (valid < kTileRows) {  // the ragged last tile: fake (clamped) streamed rows give 0
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        if (64 * h + e >= valid) pr[e] = 0.f;
                 }
             }
             if (KV) {  // P^T for dV += P^T dO
@@ -339,17 +353,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             ptx::tc_fence_after();
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
+                // 32 columns at a time: 13 warps leave 128 registers a thread, and P is live
                 uint32_t dv[32];
                 ptx::tmem_ld32(x2 + 32 * g, dv);
                 ptx::tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int e0 = 32 * g + 2 * e;
-                    const float d0 = KV ? col_d[e0] : row_d, d1 = KV ? col_d[e0 + 1] : row_d;
-                    const float s0 = pr[e0] * (__uint_as_float(dv[2 * e]) - d0);
-                    const float s1 = pr[e0 + 1] * (__uint_as_float(dv[2 * e + 1]) - d1);
-                    pk[e] = ptx::pack_bf16x2(s0, s1);
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int e0 = 32 * g + 8 * e4;
+                    float dcol[8];
+                    if (KV) {  // key-major: each column's D, four at a time
+                        const float4 a = reinterpret_cast<const float4*>(col_d)[e0 / 4];
+                        const float4 b = reinterpret_cast<const float4*>(col_d)[e0 / 4 + 1];
+                        dcol[0] = a.x; dcol[1] = a.y; dcol[2] = a.z; dcol[3] = a.w;
+                        dcol[4] = b.x; dcol[5] = b.y; dcol[6] = b.z; dcol[7] = b.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dcol[e] = row_d;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 8 * e4 + 2 * e;  // column inside this 32-column chunk
+                        const float s0 = pr[32 * g + c] * (__uint_as_float(dv[c]) - dcol[2 * e]);
+                        const float s1 = pr[32 * g + c + 1] * (__uint_as_float(dv[c + 1]) - dcol[2 * e + 1]);
+                        pk[4 * e4 + e] = ptx::pack_bf16x2(s0, s1);
+                    }
                 }
                 ptx::tmem_st16(x2 + 16 * g, pk);
             }
