@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             // Each half of the key tile is released to the tensor core as soon as it is stored,
             // so O += P V on the first half overlaps the exponentials of the second.
             const float neg = -m_run * sl2;
-            float sum0 = 0.f, sum1 = 0.f;
+            float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;  // four short addition chains
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 uint32_t pk[16];
@@ -386,8 +386,13 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                         p0 = ptx::ex2_approx(x0);
                         p1 = ptx::ex2_approx(x1);
                     }
-                    sum0 += p0;
-                    sum1 += p1;
+                    if (e & 1) {
+                        sum2 += p0;
+                        sum3 += p1;
+                    } else {
+                        sum0 += p0;
+                        sum1 += p1;
+                    }
                     pk[e] = ptx::pack_bf16x2(p0, p1);
                 }
                 ptx::tmem_st16(s_addr + 16 * g, pk);
@@ -415,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 }
             }
             if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
-            l_run = l_run * alpha + (sum0 + sum1);
+            l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
         }
         if (ok && ptx::mbar_wait(bar(C::B_OFULL), 0, abort, lim)) {
             ptx::tc_fence_after();
