@@ -357,6 +357,50 @@ def run_ours(args):
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the dense comparison")
 
+    # The pages' explicit pipeline (方法步骤详情: rearrange into P^2 subsequences, dense attention on
+    # each, rearrange back), built from this library's standalone kernels, against the fused
+    # kernel on the unpadded 768p latent (P = 2), where the two give identical results: what
+    # folding the rearranges into the attention kernel buys.
+    mat = None
+    if not args.no_materialized and rank == 0:
+        wm = synth.WORKLOADS["768p"]
+        qm, km, vm = (t.to(dev) for t in synth.qkv(wm))
+        om = torch.empty_like(qm)
+        ys = [torch.empty(fps.rearranged_shape(qm.shape, wm.P), dtype=torch.bfloat16, device=dev)
+              for _ in range(4)]
+        n = ys[0].shape[1]
+        grid = (wm.B * wm.P * wm.P, 1, 1, n, wm.heads, wm.d)
+
+        def explicit(m):
+            for x, y in zip((qm, km, vm), ys):
+                fps.skiparse_rearrange(x, wm.P, m, out=y)
+            fps.skiparse2d_attn_fwd(*(y.view(grid) for y in ys[:3]), 1, 0, out=ys[3].view(grid))
+            fps.skiparse_unrearrange(ys[3], qm.shape, wm.P, m, out=om)
+
+        def fused(m):
+            fps.skiparse2d_attn_fwd(qm, km, vm, wm.P, m, out=om)
+
+        res = {}
+        for name, fn in (("fused", fused), ("explicit", explicit)):
+            for i in range(2):
+                fn(modes[i % len(modes)])
+            m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            m0.record(stream)
+            for i in range(args.materialized_steps):
+                fn(modes[i % len(modes)])
+            m1.record(stream)
+            torch.cuda.synchronize(dev)
+            res[name] = m0.elapsed_time(m1) / args.materialized_steps
+        if fps.get_device_status() != 0:
+            raise SystemExit("device status error in the explicit-pipeline timing")
+        mat = {"workload": describe(wm) + ", no padding", "ms_fused": round(res["fused"], 3),
+               "ms_explicit": round(res["explicit"], 3),
+               "explicit_steps": "3 x skiparse_rearrange + dense (P=1) attention over B*P^2 "
+                                 "subsequences + skiparse_unrearrange",
+               "fusion_speedup": round(res["explicit"] / res["fused"], 3),
+               "hbm_bytes_saved_per_call": 2 * (4 * qm.numel() + 4 * ys[0].numel())}
+        del qm, km, vm, om, ys
+
     # Skiparse-1D (the flattened-sequence variant) at the same shape on the same kernels: the
     # 1D-vs-2D comparison, by the same padded FLOP formula with N = T * Lp
     one_d = None
@@ -486,6 +530,7 @@ def run_ours(args):
             "ms_per_layer": {k_: round(v_, 3) for k_, v_ in by_mode.items()},
             "tflops_real_pairs": real,
             "dense_p1": dense,
+            "explicit_pipeline": mat,
             "skiparse1d": one_d,
             "rearrange_kernels": rearr,
             "backward": bwd,
@@ -635,6 +680,9 @@ def main(argv=None):
     ap.add_argument("--no-rearrange", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-1d", action="store_true", help="skip the Skiparse-1D comparison")
+    ap.add_argument("--no-materialized", action="store_true",
+                    help="skip the explicit rearrange / dense / unrearrange pipeline comparison")
+    ap.add_argument("--materialized-steps", type=int, default=4)
     ap.add_argument("--one-d-steps", type=int, default=4)
     ap.add_argument("--backward-steps", type=int, default=4)
     ap.add_argument("--rearrange-steps", type=int, default=10)
