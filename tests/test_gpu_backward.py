@@ -41,7 +41,8 @@ def check_grad(got, want, what):
 
 SMALL = [synth.WORKLOADS["tiny"], synth.WORKLOADS["anyres"], synth.custom(2, 3, 13, 22, 3, 64, 2, "b2_ragged"),
          synth.custom(1, 2, 20, 30, 2, 128, 3, "p3_unequal"), synth.custom(1, 5, 16, 16, 2, 128, 1, "dense_p1"),
-         synth.custom(1, 6, 24, 40, 2, 128, 2, "multi_tile"), synth.custom(1, 1, 1, 1, 1, 64, 2, "one_token")]
+         synth.custom(1, 6, 24, 40, 2, 128, 2, "multi_tile"), synth.custom(1, 1, 1, 1, 1, 64, 2, "one_token"),
+         synth.custom(1, 2, 26, 31, 1, 64, 5, "p5"), synth.custom(1, 1, 70, 65, 1, 32, 8, "p8")]
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)

@@ -40,6 +40,10 @@ SMALL = [
     synth.custom(1, 6, 24, 40, 2, 128, 2, "multi_tile"),       # n_c = 1440: 12 tiles
     synth.custom(1, 4, 9, 33, 2, 128, 2, "thin"),              # W >> H, ragged both ways
     synth.custom(3, 2, 6, 10, 5, 64, 2, "b3_h5"),              # B = 3, 5 heads
+    synth.custom(1, 2, 26, 31, 1, 64, 5, "p5"),                # P = 5: 25 classes, padded 50x50
+    synth.custom(1, 2, 40, 45, 2, 128, 6, "p6"),               # P = 6: padded 72x72, 2 tiles
+    synth.custom(1, 1, 50, 100, 1, 64, 7, "p7"),               # P = 7: padded 98x147, H != W
+    synth.custom(1, 1, 70, 65, 1, 32, 8, "p8"),                # P = 8 (the maximum): 64 classes
 ]
 
 LARGE = ["480p", "720p", "768p", "768p_p3", "768p_p1"]
@@ -103,6 +107,23 @@ def test_rearrange_bit_exact(fps, name, mode):
     got = y.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(got, want)
     # inverse: back to the original, bit for bit
+    back = torch.empty_like(xd)
+    back.view(torch.int16).fill_(-1)
+    fps.skiparse_unrearrange(y, x.shape, w.P, mode, out=back)
+    assert torch.equal(back.view(torch.int16).cpu(), x.view(torch.int16))
+
+
+@pytest.mark.parametrize("w", [w for w in SMALL if w.P >= 5], ids=lambda w: w.name)
+@pytest.mark.parametrize("mode", [TOK, GRP])
+def test_rearrange_bit_exact_large_p(fps, w, mode):
+    """P = 5..8 (up to 64 classes, most of them holding pad slots) on small latents."""
+    x, _, _ = synth.qkv(w)
+    want = oracle.rearrange(x, w.P, mode)
+    xd = x.cuda()
+    y = torch.empty(fps.rearranged_shape(x.shape, w.P), dtype=torch.bfloat16, device="cuda")
+    y.view(torch.int16).fill_(-1)
+    fps.skiparse_rearrange(xd, w.P, mode, out=y)
+    assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), want)
     back = torch.empty_like(xd)
     back.view(torch.int16).fill_(-1)
     fps.skiparse_unrearrange(y, x.shape, w.P, mode, out=back)

@@ -116,7 +116,8 @@ def test_class_maps_golden():
 
 
 @pytest.mark.parametrize("T,Hp,Wp,P,C", [(1, 4, 4, 2, 3), (2, 8, 12, 2, 5), (2, 9, 18, 3, 2),
-                                         (1, 16, 16, 4, 1), (3, 6, 5, 1, 2)])
+                                         (1, 16, 16, 4, 1), (3, 6, 5, 1, 2), (1, 25, 50, 5, 1),
+                                         (1, 64, 64, 8, 1)])
 def test_token_wise_is_pixel_unshuffle(T, Hp, Wp, P, C):
     """核心方法: token-wise rearrange is pixel unshuffle (torch's library routine)."""
     x = torch.randint(0, 60000, (1, T, Hp, Wp, 1, C), dtype=torch.int32)
@@ -130,7 +131,7 @@ def test_token_wise_is_pixel_unshuffle(T, Hp, Wp, P, C):
 
 
 @pytest.mark.parametrize("T,Hp,Wp,P,C", [(1, 4, 4, 2, 3), (2, 8, 12, 2, 2), (1, 9, 18, 3, 2),
-                                         (1, 16, 32, 4, 1)])
+                                         (1, 16, 32, 4, 1), (1, 25, 50, 5, 1), (1, 64, 128, 8, 1)])
 def test_group_wise_is_patch_unshuffle(T, Hp, Wp, P, C):
     """核心方法: group-wise is patch unshuffle: fold each P x P patch into channels
     (pixel_unshuffle), distribute the patch grid the pixel-unshuffle way
@@ -259,7 +260,8 @@ def test_p1_is_full_attention(T, H, W, heads, d):
 
 BRUTE_CASES = [synth.WORKLOADS["tiny"], synth.WORKLOADS["anyres"],
                synth.custom(2, 2, 5, 7, 2, 8, 3), synth.custom(1, 1, 3, 17, 1, 4, 4),
-               synth.custom(1, 2, 6, 6, 2, 16, 1)]
+               synth.custom(1, 2, 6, 6, 2, 16, 1), synth.custom(1, 1, 26, 31, 1, 8, 5),
+               synth.custom(1, 1, 20, 23, 1, 4, 8)]
 
 
 @pytest.mark.parametrize("w", BRUTE_CASES, ids=lambda w: w.name + f"_P{w.P}_H{w.H}W{w.W}")
