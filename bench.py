@@ -56,6 +56,8 @@ KNOWN_TRAFFIC = {
     "5d623923e1bf3aa7": 3.086e9,
     # the kernel with four row-sum chains, the same capture: 2.33 GB read + 0.757 GB written
     "1e3835ddabab1731": 3.087e9,
+    # softmax waits made warp-uniform, the same capture: 2.33 GB read + 0.756 GB written
+    "e17da04fa61e70d2": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",

@@ -287,13 +287,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         for (int j = 0; j < nstream; ++j) {
             const int s = j & 1;
             const int valid = n_c - j * kTileRows;     // streamed rows in this tile (>= 1)
-            if (!ptx::mbar_wait(bar(C::B_X1), j & 1, abort, lim)) {
+            // every wait of a softmax warp is made uniform over the warp: the tcgen05.ld/st below
+            // are .sync.aligned and need all 32 lanes
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_X1), j & 1, abort, lim))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
             // the L/D vectors were written by the producers' cp.async: observe their barrier too
-            if (!ptx::mbar_wait(KV ? bar(C::B_FULL + s) : bar(C::B_STAT), KV ? (j >> 1) & 1 : 0, abort, lim)) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(KV ? bar(C::B_FULL + s) : bar(C::B_STAT),
+                                                        KV ? (j >> 1) & 1 : 0, abort, lim))) {
                 ok = false;
                 break;
             }
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(C::B_P));
             }
-            if (!ptx::mbar_wait(bar(C::B_X2), j & 1, abort, lim)) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_X2), j & 1, abort, lim))) {
                 ok = false;
                 break;
             }
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar(C::B_DS));
         }
-        if (ok && ptx::mbar_wait(bar(C::B_ACC), 0, abort, lim)) {
+        if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_ACC), 0, abort, lim))) {
             ptx::tc_fence_after();
             const int si = first + row;                 // stationary row (key or query)
             const size_t grow = si < n_c ? static_cast<size_t>(rows(si)) : 0;

@@ -319,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         bool ok = true;
         if (SKIPARSE_MUFU_TURNS && qt == 1) ptx::mbar_arrive(bar(C::B_TURN + 0));  // tile 0 goes first
         for (int j = 0; j < nkv; ++j) {
-            if (!ptx::mbar_wait(sfull, j & 1, abort, lim)) {
+            // Every wait of a softmax warp is made uniform over the warp (a lane can see the abort
+            // flag while another sees the phase complete): the tcgen05.ld/st below are
+            // .sync.aligned and need all 32 lanes.
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(sfull, j & 1, abort, lim))) {
                 ok = false;
                 break;
             }
@@ -362,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
                 m_run = mx;
             }
-            if (SKIPARSE_MUFU_TURNS && !ptx::mbar_wait(my_turn, j & 1, abort, lim)) {
+            if (SKIPARSE_MUFU_TURNS && !__all_sync(0xffffffffu, ptx::mbar_wait(my_turn, j & 1, abort, lim))) {
                 ok = false;
                 break;
             }
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
             l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
         }
-        if (ok && ptx::mbar_wait(bar(C::B_OFULL), 0, abort, lim)) {
+        if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_OFULL), 0, abort, lim))) {
             ptx::tc_fence_after();
             const int qi = q_first + qt * kBM + row;
             const float inv_l = 1.f / l_run;
