@@ -530,6 +530,8 @@ def run_ours(args):
             "gpu_launches": args.steps,
             "clocks": clk,
             "ms_per_layer": {k_: round(v_, 3) for k_, v_ in by_mode.items()},
+            "ms_per_launch": {"median": round(statistics.median(per_launch), 3),
+                              "min": round(min(per_launch), 3)},
             "tflops_real_pairs": real,
             "dense_p1": dense,
             "explicit_pipeline": mat,
