@@ -23,6 +23,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "attn_common.cuh"
 
 namespace skiparse {
@@ -460,15 +462,17 @@ __global__ void __launch_bounds__(256) skiparse_bwd_delta_kernel(const uint16_t*
 template <int D, bool KV>
 int launch_bwd_d(const BwdParams& p, const Geometry& g, cudaStream_t stream) {
     using C = BwdCfg<D, KV>;
-    static int attr_done_dev[64] = {0};
+    // per device: the kernel's shared-memory attribute is set (host threads may race here;
+    // setting it twice is harmless, the flag only has to be a race-free read)
+    static std::atomic<int> attr_done_dev[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return static_cast<int>(e);
-    if (dev >= 0 && dev < 64 && !attr_done_dev[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done_dev[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(skiparse_attn_bwd_kernel<D, KV>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return static_cast<int>(e);
-        attr_done_dev[dev] = 1;
+        attr_done_dev[dev].store(1, std::memory_order_release);
     }
     int n_max = 0;
     for (int ci = 0; ci < g.Ph; ++ci)

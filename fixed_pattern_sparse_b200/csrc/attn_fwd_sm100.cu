@@ -29,6 +29,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "attn_common.cuh"
 
 namespace skiparse {
@@ -469,11 +471,13 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
 template <int D>
 int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
     using C = Cfg<D>;
-    static int attr_done_dev[64] = {0};
+    // per device: the kernel's shared-memory attribute is set (host threads may race here;
+    // setting it twice is harmless, the flag only has to be a race-free read)
+    static std::atomic<int> attr_done_dev[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return static_cast<int>(e);
-    if (dev >= 0 && dev < 64 && !attr_done_dev[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_done_dev[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(skiparse_attn_fwd_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return static_cast<int>(e);
@@ -485,7 +489,7 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
             if (e != cudaSuccess) return static_cast<int>(e);
             if (fa.numRegs != kLaunchRegs) return static_cast<int>(cudaErrorInvalidConfiguration);
         }
-        attr_done_dev[dev] = 1;
+        attr_done_dev[dev].store(1, std::memory_order_release);
     }
     int n_max = 0;
     for (int ci = 0; ci < g.Ph; ++ci)
