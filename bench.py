@@ -58,6 +58,9 @@ KNOWN_TRAFFIC = {
     "1e3835ddabab1731": 3.087e9,
     # softmax waits made warp-uniform, the same capture: 2.33 GB read + 0.756 GB written
     "e17da04fa61e70d2": 3.086e9,
+    # host-side attribute flags made atomics (device code unchanged), the same capture:
+    # 2.33 GB read + 0.756 GB written
+    "26bde2fce291ecaa": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
