@@ -61,6 +61,9 @@ KNOWN_TRAFFIC = {
     # host-side attribute flags made atomics (device code unchanged), the same capture:
     # 2.33 GB read + 0.756 GB written
     "26bde2fce291ecaa": 3.086e9,
+    # row-bound checks added for the debug build (compiled out here), the same capture:
+    # 2.33 GB read + 0.756 GB written
+    "f28ade9892c14eb0": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",

@@ -11,6 +11,9 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libskiparse.so")
+# The bounds-checking debug build of the same library (SKIPARSE_DEBUG=1), for tests and for
+# hunting an out-of-range access: `python -m fixed_pattern_sparse_b200.build --debug`.
+DEBUG_LIB_PATH = os.path.join(HERE, "libskiparse_debug.so")
 
 # Every symbol include/skiparse.h declares, with (restype, argtypes).
 _I, _LL, _ULL, _VP, _CP = ctypes.c_int, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_void_p, ctypes.c_char_p
@@ -32,6 +35,7 @@ SIGNATURES = {
     "skiparse_last_error_string": (_CP, []),
     "skiparse_set_wait_limit_ns": (_ULL, [_ULL]),
     "skiparse_debug_inject_fault": (_I, [_I]),
+    "skiparse_debug_shrink_bounds": (_I, [_LL]),
     "skiparse_debug_exp2": (_I, [_VP, _VP, _LL, _I, _VP]),
     "skiparse1d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse1d_attn_fwd_lse": (_I, [_VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
@@ -49,7 +53,8 @@ SIGNATURES = {
 }
 
 STATUS = {0: "SKIPARSE_OK", 1: "SKIPARSE_ERR_INVALID_ARG", 2: "SKIPARSE_ERR_UNSUPPORTED",
-          3: "SKIPARSE_ERR_MISALIGNED", 4: "SKIPARSE_ERR_CUDA", 5: "SKIPARSE_ERR_TIMEOUT"}
+          3: "SKIPARSE_ERR_MISALIGNED", 4: "SKIPARSE_ERR_CUDA", 5: "SKIPARSE_ERR_TIMEOUT",
+          6: "SKIPARSE_ERR_BOUNDS"}
 
 
 class SkiparseError(RuntimeError):
@@ -61,20 +66,33 @@ class SkiparseError(RuntimeError):
 _LIB = None
 
 
+_DEBUG_LIB = None
+
+
+def _load(path: str, how: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `{how}` (there is no CPU or library fallback)")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
 def lib() -> ctypes.CDLL:
     global _LIB
     if _LIB is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(
-                f"{LIB_PATH} is missing: build it with `python -m fixed_pattern_sparse_b200.build` "
-                "(there is no CPU or library fallback)")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.restype = res
-            fn.argtypes = args
-        _LIB = L
+        _LIB = _load(LIB_PATH, "python -m fixed_pattern_sparse_b200.build")
     return _LIB
+
+
+def debug_lib() -> ctypes.CDLL:
+    """The bounds-checking debug build, bound like lib() (separate library, separate state)."""
+    global _DEBUG_LIB
+    if _DEBUG_LIB is None:
+        _DEBUG_LIB = _load(DEBUG_LIB_PATH, "python -m fixed_pattern_sparse_b200.build --debug")
+    return _DEBUG_LIB
 
 
 def check(code: int, what: str) -> None:

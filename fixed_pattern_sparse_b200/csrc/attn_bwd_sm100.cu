@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         // pair 1 (warps 10-11) the second; within a pair, warp pw copies rows [64pw, 64pw+64).
         const int pair = (warp - kBwdProd0) >> 1;
         const int pw = (warp - kBwdProd0) & 1;
-        const TileRows ta = tile_rows(rows, first, n_c, pw, lane);
+        const TileRows ta = tile_rows(rows, first, n_c, pw, lane, p.nrows, p.status);
         load_tile_rows<D>(sbase + (pair ? C::OFF_A2 : C::OFF_A1), pair ? g_a2 : g_a1, ta, pw, lane);
         if (!KV && pair == 0) {  // the stationary queries' L and D
             load_vec(sbase + C::OFF_VEC, p.lse, ta, pw, lane);
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 }
             }
             const uint32_t slot = sbase + C::OFF_B + 2 * s * C::TILE_BYTES;
-            const TileRows tr = tile_rows(rows, j * kTileRows, n_c, pw, lane);
+            const TileRows tr = tile_rows(rows, j * kTileRows, n_c, pw, lane, p.nrows, p.status);
             load_tile_rows<D>(slot + (pair ? C::TILE_BYTES : 0), pair ? g_b2 : g_b1, tr, pw, lane);
             if (KV && pair == 0) {  // the streamed queries' L and D
                 const uint32_t v = sbase + C::OFF_VEC + s * 2 * 4 * kTileRows;
@@ -393,7 +393,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_ACC), 0, abort, lim))) {
             ptx::tc_fence_after();
             const int si = first + row;                 // stationary row (key or query)
-            const size_t grow = si < n_c ? static_cast<size_t>(rows(si)) : 0;
+            const bool store = si < n_c && row_ok(rows(si), p.nrows, p.status);
+            const size_t grow = store ? static_cast<size_t>(rows(si)) : 0;
             constexpr int HALF = D / 2;                 // accumulator columns of this warpgroup
             // key-major: acc1 = dV (unscaled), acc2 = dK ; query-major: acc1 = dQ
 #pragma unroll
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         pk[e] = ptx::pack_bf16x2(__uint_as_float(av[2 * e]) * mul, __uint_as_float(av[2 * e + 1]) * mul);
-                    if (si < n_c) {
+                    if (store) {
                         uint4* dst = reinterpret_cast<uint4*>(out + grow * D + HALF * h + 16 * g);
                         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);

@@ -107,15 +107,18 @@ __device__ __forceinline__ void fence_proxy_async() {
 
 // The two token rows a producer lane copies for tile rows [first, first+128) of the class's
 // real-token list: tile rows 64*pw + lane and 64*pw + lane + 32 (rows past n_c repeat row
-// n_c-1; they are masked or never stored). K and V tiles of one key step share them.
+// n_c-1; they are masked or never stored). K and V tiles of one key step share them. nrows and
+// status serve the debug build's bounds check (the tensor's row count, the error word).
 struct TileRows {
     int ra, rb;
 };
-__device__ __forceinline__ TileRows tile_rows(const RowMap& rows, int first, int n_c, int pw, int lane) {
+__device__ __forceinline__ TileRows tile_rows(const RowMap& rows, int first, int n_c, int pw, int lane,
+                                              long long nrows, int* status) {
     int ia = first + 64 * pw + lane, ib = ia + 32;
     ia = ia < n_c ? ia : n_c - 1;
     ib = ib < n_c ? ib : n_c - 1;
-    return TileRows{rows(ia), rows(ib)};
+    return TileRows{static_cast<int>(load_row(rows(ia), nrows, status)),
+                    static_cast<int>(load_row(rows(ib), nrows, status))};
 }
 
 // Issues the cp.async copies of a 128-row tile whose token rows tile_rows() gave into the
@@ -148,8 +151,9 @@ __device__ __forceinline__ void load_tile_rows(uint32_t dst, const uint16_t* __r
 // tile_rows + load_tile_rows for a tile loaded from one tensor only.
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const uint16_t* __restrict__ g,
-                                          const RowMap& rows, int first, int n_c, int pw, int lane) {
-    load_tile_rows<D>(dst, g, tile_rows(rows, first, n_c, pw, lane), pw, lane);
+                                          const RowMap& rows, int first, int n_c, int pw, int lane,
+                                          long long nrows, int* status) {
+    load_tile_rows<D>(dst, g, tile_rows(rows, first, n_c, pw, lane, nrows, status), pw, lane);
 }
 
 

@@ -177,8 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         // they have landed, so a tile is released as soon as it is in shared memory.
         const int pw = warp - kProdWarp0;
         const int fault_skip = (p.fault == 1 && pw == 0 && lane == 0);
-        load_tile<D>(sbase + C::OFF_Q, p.q, rows, q_first, n_c, pw, lane);
-        load_tile<D>(sbase + C::OFF_Q + C::TILE_BYTES, p.q, rows, q_first + kBM, n_c, pw, lane);
+        load_tile<D>(sbase + C::OFF_Q, p.q, rows, q_first, n_c, pw, lane, p.nrows, p.status);
+        load_tile<D>(sbase + C::OFF_Q + C::TILE_BYTES, p.q, rows, q_first + kBM, n_c, pw, lane, p.nrows,
+                     p.status);
         cp_async_arrive_noinc(bar(C::B_Q));
         bool ok = true;
         TileRows kv{0, 0};  // token rows of key step j, shared by its K and V tiles
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             const bool is_v = L & 1;
             const int nst = is_v ? C::VST : C::KST;
             const int s = j % nst;
-            if (!is_v) kv = tile_rows(rows, j * kBN, n_c, pw, lane);
+            if (!is_v) kv = tile_rows(rows, j * kBN, n_c, pw, lane, p.nrows, p.status);
             if (j >= nst) {
                 const int empty = (is_v ? C::B_VEMPTY : C::B_KEMPTY) + s;
                 int w_ok = 1;
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             const int qi = q_first + qt * kBM + row;
             const float inv_l = 1.f / l_run;
             uint4* dst = nullptr;
-            if (qi < n_c) {
+            if (qi < n_c && row_ok(rows(qi), p.nrows, p.status)) {
                 const int grow = rows(qi);
                 dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(grow) * D);
                 // log-sum-exp (natural log) of the scaled scores: m*log2(e)/sqrt(d) + log2(l), in ln

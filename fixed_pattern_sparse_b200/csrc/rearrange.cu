@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(kThreads) skiparse_rearrange_kernel(const Rear
             const long long seq = static_cast<long long>(b) * q2 + ci * p.Pw + cj;
             src_row = seq * p.n + (static_cast<long long>(t) * p.R + r) * p.S + s;
         }
-        const uint4* s_row = src + src_row * p.row_chunks;
+        if (real && !row_ok(src_row, p.src_rows, p.status)) real = false;  // debug builds
+        const uint4* s_row = src + (real ? src_row : 0) * p.row_chunks;
         uint4* d_row = dst + row * p.row_chunks;
         for (int k = lane; k < p.row_chunks; k += 32 * kUnroll) {
             uint4 v[kUnroll];

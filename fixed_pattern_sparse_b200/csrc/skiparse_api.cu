@@ -26,6 +26,15 @@ int cuda_fail(int err) {
     return SKIPARSE_ERR_CUDA;
 }
 std::atomic<int> g_fault{0};
+// Debug builds: rows by which the next launch's bounds are declared smaller than its tensors
+// (skiparse_debug_shrink_bounds), so that a test sees the bounds check report without any
+// access leaving a tensor. Consumed by the next launch.
+std::atomic<long long> g_bounds_shrink{0};
+
+long long checked_bound(long long rows) {
+    const long long shrink = g_bounds_shrink.exchange(0);
+    return SKIPARSE_DEBUG ? rows - shrink : rows;
+}
 
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
@@ -108,11 +117,15 @@ const char* skiparse_status_string(int status) {
         case SKIPARSE_ERR_MISALIGNED: return "SKIPARSE_ERR_MISALIGNED";
         case SKIPARSE_ERR_CUDA: return "SKIPARSE_ERR_CUDA";
         case SKIPARSE_ERR_TIMEOUT: return "SKIPARSE_ERR_TIMEOUT";
+        case SKIPARSE_ERR_BOUNDS: return "SKIPARSE_ERR_BOUNDS";
         default: return "SKIPARSE_ERR_UNKNOWN";
     }
 }
 
-const char* skiparse_version(void) { return "skiparse-b200 0.1 (sm_100a, tcgen05)"; }
+const char* skiparse_version(void) {
+    return SKIPARSE_DEBUG ? "skiparse-b200 0.1 (sm_100a, tcgen05; debug build: row bounds checked)"
+                          : "skiparse-b200 0.1 (sm_100a, tcgen05)";
+}
 
 const char* skiparse_last_error_string(void) { return t_last_cuda_error; }
 
@@ -171,6 +184,13 @@ unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns) {
 int skiparse_debug_inject_fault(int kind) {
     if (kind != 0 && kind != 1) return SKIPARSE_ERR_INVALID_ARG;
     g_fault.store(kind);
+    return SKIPARSE_OK;
+}
+
+int skiparse_debug_shrink_bounds(long long rows) {
+    if (!SKIPARSE_DEBUG) return SKIPARSE_ERR_UNSUPPORTED;
+    if (rows < 0) return SKIPARSE_ERR_INVALID_ARG;
+    g_bounds_shrink.store(rows);
     return SKIPARSE_OK;
 }
 
@@ -240,6 +260,7 @@ static int attn_fwd_common(int dims, const void* q, const void* k, const void* v
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.exchange(0);
+    p.nrows = checked_bound(rows);
     const int e = skiparse::launch_attn_fwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
@@ -314,6 +335,7 @@ static int attn_bwd_common(int dims, const void* q, const void* k, const void* v
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     p.wait_limit_ns = g_wait_limit_ns.load();
+    p.nrows = checked_bound(rows);
     const int e = skiparse::launch_attn_bwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
@@ -357,6 +379,9 @@ static int rearrange_common(int dims, const void* src, void* dst, int B, int T, 
     p.n = g.n;
     p.row_chunks = static_cast<int>(row_bytes / 16);
     p.nrows = kind == 1 ? ntok : nslot;
+    p.src_rows = checked_bound(kind == 0 ? ntok : nslot);
+    p.status = status_ptr();
+    if (!p.status) return SKIPARSE_ERR_CUDA;
     const int e = skiparse::launch_rearrange(p, kind, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }

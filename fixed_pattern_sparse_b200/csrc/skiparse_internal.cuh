@@ -24,6 +24,15 @@
 
 namespace skiparse {
 
+// Debug build (SKIPARSE_DEBUG=1, libskiparse_debug.so): every token row index a kernel computes
+// for a global load or store is checked against the row count of its tensor. An index outside
+// is recorded as kErrBounds in the device status word and never used: a load reads row 0
+// instead, a store is dropped. No access leaves its tensor, so the check cannot itself fault.
+// Release builds compile the checks out.
+#ifndef SKIPARSE_DEBUG
+#define SKIPARSE_DEBUG 0
+#endif
+
 constexpr int kMaxP = 8;
 constexpr int kMaxAxisClasses = kMaxP * kMaxP;  // Skiparse-1D: P^2 classes on one axis
 
@@ -67,6 +76,7 @@ struct AttnParams {
     float scale_log2;              // log2(e)/sqrt(d)
     unsigned long long wait_limit_ns;
     int fault;                     // test hook: 1 = one producer never signals the first K tile
+    long long nrows;               // (token, head) rows of q, k, v, out, lse: the debug bound
 };
 
 // Parameters of the backward kernels.
@@ -87,6 +97,7 @@ struct BwdParams {
     float scale_log2;              // log2(e)/sqrt(d)
     float scale;                   // 1/sqrt(d)
     unsigned long long wait_limit_ns;
+    long long nrows;               // (token, head) rows of every tensor above: the debug bound
 };
 
 struct RearrangeParams {
@@ -96,10 +107,36 @@ struct RearrangeParams {
     long long n;          // padded subsequence length
     int row_chunks;       // 16-byte chunks per token row (heads*d*2/16)
     long long nrows;      // rows to write: B*P*P*n (rearrange, switch) or B*T*H*W (unrearrange)
+    long long src_rows;   // token rows of the source tensor: the debug bound
+    int* status;          // device error word
 };
 
 // Status codes (mirror include/skiparse.h).
-enum : int { kOk = 0, kErrTimeout = 5 };
+enum : int { kOk = 0, kErrTimeout = 5, kErrBounds = 6 };
+
+// The row index a global load may use: `row` itself, or (debug builds, row outside
+// [0, nrows)) row 0 after recording kErrBounds.
+__device__ __forceinline__ long long load_row(long long row, long long nrows, int* status) {
+#if SKIPARSE_DEBUG
+    if (row < 0 || row >= nrows) {
+        atomicExch(status, kErrBounds);
+        return 0;
+    }
+#endif
+    return row;
+}
+
+// Whether a global access may use row index `row` (debug builds: false, after recording
+// kErrBounds, when it lies outside [0, nrows)); the caller then skips the access.
+__device__ __forceinline__ bool row_ok(long long row, long long nrows, int* status) {
+#if SKIPARSE_DEBUG
+    if (row < 0 || row >= nrows) {
+        atomicExch(status, kErrBounds);
+        return false;
+    }
+#endif
+    return true;
+}
 
 // Launchers (defined in the kernel translation units). They return the cudaError_t as int.
 int launch_attn_fwd(const AttnParams& p, const Geometry& g, void* stream);

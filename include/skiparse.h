@@ -55,7 +55,9 @@ enum {
     SKIPARSE_ERR_UNSUPPORTED = 2, /* valid but outside the supported set (d, P, size) */
     SKIPARSE_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
     SKIPARSE_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor map) */
-    SKIPARSE_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired; its output is invalid */
+    SKIPARSE_ERR_TIMEOUT = 5,     /* a kernel's bounded wait expired; its output is invalid */
+    SKIPARSE_ERR_BOUNDS = 6       /* debug build only: a kernel computed a token row outside its
+                                     tensor; the access was skipped and the output is invalid */
 };
 
 /*
@@ -255,7 +257,8 @@ SKIPARSE_API long long skiparse1d_rearranged_numel(int B, int T, int H, int W, i
 /*
  * Synchronizes `stream`, then returns and clears the current device's error word: SKIPARSE_OK,
  * or SKIPARSE_ERR_TIMEOUT if any kernel since the last call gave up on a bounded wait (its
- * output is then invalid), or SKIPARSE_ERR_CUDA if the synchronization itself failed.
+ * output is then invalid), or SKIPARSE_ERR_BOUNDS (debug build only) if a kernel computed a
+ * token row outside its tensor, or SKIPARSE_ERR_CUDA if the synchronization itself failed.
  */
 SKIPARSE_API int skiparse_get_device_status(skiparse_stream_t stream);
 
@@ -284,6 +287,19 @@ SKIPARSE_API unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns
  * Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
  */
 SKIPARSE_API int skiparse_debug_inject_fault(int kind);
+
+/*
+ * Debug build (libskiparse_debug.so, compiled with SKIPARSE_DEBUG=1; no counterpart on the
+ * pages). Its kernels check every token row index they compute for a global load or store
+ * against the row count of the tensor; an index outside is recorded as SKIPARSE_ERR_BOUNDS in
+ * the device error word and the access is skipped (a load reads row 0, a store is dropped),
+ * so the check itself never leaves a tensor. This hook declares the next launch's row counts
+ * `rows` smaller than the tensors really are, so that a test can see the check report while
+ * every actual access stays inside the tensors. Consumed by the next launch of any entry point.
+ * Returns SKIPARSE_OK (debug build), SKIPARSE_ERR_UNSUPPORTED (release build, which has no
+ * checks) or SKIPARSE_ERR_INVALID_ARG (rows < 0).
+ */
+SKIPARSE_API int skiparse_debug_shrink_bounds(long long rows);
 
 /*
  * Diagnostic (no counterpart on the pages): y[i] = 2^x[i] for n fp32 device values, evaluated

@@ -185,3 +185,19 @@ def test_host_entry_rejects_bad_arguments_synchronously(L):
     over = (FAKE, FAKE + big, FAKE + 2 * big, FAKE + 64, 1, 2, 8, 8, 4, 32, 2, 0)       # out overlaps q
     assert L.skiparse2d_attn_fwd_host(*over, 2, FAKE + 4 * big, need, None) == 1
     assert L.skiparse1d_attn_fwd_host(*args, 2, FAKE + 4 * big, need - 1, None) == 1
+
+
+def test_debug_build_hook_and_exports():
+    """The bounds-checking debug build exports the same C ABI; only it accepts the hook that
+    declares the next launch's bounds smaller (the release build has no checks)."""
+    from fixed_pattern_sparse_b200 import _lib
+    R = _lib.lib()
+    assert R.skiparse_debug_shrink_bounds(3) == 2  # SKIPARSE_ERR_UNSUPPORTED
+    assert b"debug" not in R.skiparse_version()
+    D = _lib.debug_lib()
+    for name in _lib.SIGNATURES:
+        assert hasattr(D, name), name
+    assert b"debug" in D.skiparse_version()
+    assert D.skiparse_debug_shrink_bounds(-1) == 1
+    assert D.skiparse_debug_shrink_bounds(0) == 0
+    assert D.skiparse_status_string(6) == b"SKIPARSE_ERR_BOUNDS"
