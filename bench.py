@@ -230,7 +230,7 @@ def oracle_sample_rows(w, mode, nrows: int, group: int = 0) -> np.ndarray:
 
 def time_oracle(w, q, k, v, mode, target_s: float, nthreads: int):
     """Times the oracle on a bounded sample sized to about target_s seconds of CPU work.
-    Returns (TFLOP/s, seconds, rows, description)."""
+    Returns (TFLOP/s, seconds, description, sampled rows, the oracle's fp64 output rows)."""
     import oracle
     n_c = max(class_lens(w, mode))
     per_row = 4.0 * n_c * w.d
@@ -241,16 +241,30 @@ def time_oracle(w, q, k, v, mode, target_s: float, nthreads: int):
     nrows = int(min(max(len(rows) * target_s / max(dt, 1e-3), nthreads), 200000))
     rows = oracle_sample_rows(w, mode, nrows)
     t = time.perf_counter()
-    oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
+    want = oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
     dt = time.perf_counter() - t
     flops = per_row * len(rows)
     desc = (f"{len(rows)} query rows of one (class, head) subsequence of the {w.name} workload "
             f"({MODE_NAME[mode]}), each attending over its class's ~{n_c} real keys; the oracle's "
             f"per-subsequence gather included")
-    return flops / dt / 1e12, dt, len(rows), desc
+    return flops / dt / 1e12, dt, desc, rows, want
 
 
 MODE_NAME = synth.MODE_NAMES
+
+
+class nvtx_range:
+    """An NVTX range around one leg of the benchmark (host-side annotation for a timeline tool;
+    no effect on the device timings)."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
 
 
 # --------------------------------------------------------------------------- our arm
@@ -286,11 +300,12 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    for i in range(args.steps):
-        starts[i].record(stream)
-        step(i)
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
+    with nvtx_range("timed forward steps"):
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step(i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     barrier(world)
     clk = clocks.stop(t_wall0, t_wall1)
@@ -331,12 +346,14 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
+        torch.cuda.nvtx.range_push("end-to-end host-buffer steps")
         e0.record(stream)
         for i in range(args.e2e_steps):
             fps.attn_fwd_host(qh, kh, vh, w.P, modes[i % len(modes)], oh, heads_per_group=hg, workspace=ws,
                               stream=stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the end-to-end timing")
@@ -354,11 +371,12 @@ def run_ours(args):
         for _ in range(2):
             fps.skiparse2d_attn_fwd(qd, kd, vd, 1, 0, out=out)
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for _ in range(args.dense_steps):
-            fps.skiparse2d_attn_fwd(qd, kd, vd, 1, 0, out=out)
-        d1.record(stream)
-        torch.cuda.synchronize(dev)
+        with nvtx_range("dense P=1 steps"):
+            d0.record(stream)
+            for _ in range(args.dense_steps):
+                fps.skiparse2d_attn_fwd(qd, kd, vd, 1, 0, out=out)
+            d1.record(stream)
+            torch.cuda.synchronize(dev)
         dms = d0.elapsed_time(d1) / args.dense_steps
         dense = {"ms_per_layer_p1": round(dms, 3), "tflops_p1": round(flops_padded(wd) / (dms / 1e3) / 1e12, 1),
                  "sparse_speedup": round(dms / statistics.mean(per_launch), 3)}
@@ -389,6 +407,7 @@ def run_ours(args):
             fps.skiparse2d_attn_fwd(qm, km, vm, wm.P, m, out=om)
 
         res = {}
+        torch.cuda.nvtx.range_push("explicit pipeline vs fused, 768p")
         for name, fn in (("fused", fused), ("explicit", explicit)):
             for i in range(2):
                 fn(modes[i % len(modes)])
@@ -399,6 +418,7 @@ def run_ours(args):
             m1.record(stream)
             torch.cuda.synchronize(dev)
             res[name] = m0.elapsed_time(m1) / args.materialized_steps
+        torch.cuda.nvtx.range_pop()
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the explicit-pipeline timing")
         mat = {"workload": describe(wm) + ", no padding", "ms_fused": round(res["fused"], 3),
@@ -464,11 +484,12 @@ def run_ours(args):
         for i in range(3):
             bstep(i)
         b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        for i in range(args.backward_steps):
-            bstep(i)
-        b1.record(stream)
-        torch.cuda.synchronize(dev)
+        with nvtx_range("backward steps"):
+            b0.record(stream)
+            for i in range(args.backward_steps):
+                bstep(i)
+            b1.record(stream)
+            torch.cuda.synchronize(dev)
         bms = b0.elapsed_time(b1) / args.backward_steps
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the backward timing")
@@ -513,9 +534,18 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         nth = oracle.default_threads()
-        val, dt, nrows, desc = time_oracle(w, q, k, v, modes[0], args.cpu_seconds, nth)
+        val, dt, desc, orows, want = time_oracle(w, q, k, v, modes[0], args.cpu_seconds, nth)
+        # the same rows from the kernel (outside every timed region): the bench's own parity
+        # check against the oracle, at the tolerance of the parity tests
+        fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, modes[0], out=out)
+        got = out.reshape(-1, w.d).index_select(0, torch.from_numpy(orows).to(dev)).double().cpu().numpy()
+        err = np.abs(got - want)
         cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": nth, "kind": "oracle",
-               "sample": desc, "seconds": round(dt, 2)}
+               "sample": desc, "seconds": round(dt, 2),
+               "parity": {"rows": int(len(orows)), "max_abs_err": float(err.max()),
+                          "mean_abs_err": float(err.mean()),
+                          "ok": bool(np.isfinite(got).all() and err.max() <= 1e-2 and err.mean() <= 1e-3),
+                          "tolerance": "max <= 1e-2, mean <= 1e-3 against the fp64 oracle"}}
 
     if rank == 0:
         real = {MODE_NAME[m]: round(flops_real(w, m) / (by_mode[MODE_NAME[m]] / 1e3) / 1e12, 1)
