@@ -64,6 +64,9 @@ KNOWN_TRAFFIC = {
     # row-bound checks added for the debug build (compiled out here), the same capture:
     # 2.33 GB read + 0.756 GB written
     "f28ade9892c14eb0": 3.086e9,
+    # a backward fault-hook field in the shared parameter header, the same capture:
+    # 2.33 GB read + 0.756 GB written
+    "8686c48250f57858": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",

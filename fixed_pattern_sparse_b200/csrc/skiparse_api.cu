@@ -181,8 +181,14 @@ unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns) {
     return g_wait_limit_ns.exchange(ns == 0 ? kDefaultWaitNs : ns);
 }
 
+// A pending fault of `kind`, consumed (one launch) by the entry point it concerns only.
+static int take_fault(int kind) {
+    int expected = kind;
+    return g_fault.compare_exchange_strong(expected, 0) ? 1 : 0;
+}
+
 int skiparse_debug_inject_fault(int kind) {
-    if (kind != 0 && kind != 1) return SKIPARSE_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1 && kind != 2) return SKIPARSE_ERR_INVALID_ARG;
     g_fault.store(kind);
     return SKIPARSE_OK;
 }
@@ -259,7 +265,7 @@ static int attn_fwd_common(int dims, const void* q, const void* k, const void* v
     }
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     p.wait_limit_ns = g_wait_limit_ns.load();
-    p.fault = g_fault.exchange(0);
+    p.fault = take_fault(1);
     p.nrows = checked_bound(rows);
     const int e = skiparse::launch_attn_fwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
@@ -336,6 +342,7 @@ static int attn_bwd_common(int dims, const void* q, const void* k, const void* v
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.nrows = checked_bound(rows);
+    p.fault = take_fault(2);
     const int e = skiparse::launch_attn_bwd(p, g, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }

@@ -98,6 +98,8 @@ struct BwdParams {
     float scale;                   // 1/sqrt(d)
     unsigned long long wait_limit_ns;
     long long nrows;               // (token, head) rows of every tensor above: the debug bound
+    int fault;                     // test hook: 1 = one producer never signals the key-major
+                                   // kernel's first streamed tile
 };
 
 struct RearrangeParams {

@@ -280,11 +280,13 @@ SKIPARSE_API const char* skiparse_version(void);
 SKIPARSE_API unsigned long long skiparse_set_wait_limit_ns(unsigned long long ns);
 
 /*
- * Test hook for failure detection. kind = 1 makes the next skiparse2d_attn_fwd launch of this
- * process lose one arrival on its first K-tile barrier (one producer thread never signals it),
- * so that the consumer's bounded wait expires and the kernel reports SKIPARSE_ERR_TIMEOUT
- * without faulting or hanging the GPU. kind = 0 clears it. The hook is consumed by one launch.
- * Returns SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
+ * Test hook for failure detection. kind = 1 makes the next forward launch of this process
+ * (skiparse2d_attn_fwd and the other forward entry points) lose one arrival on its first K-tile
+ * barrier (one producer thread never signals it); kind = 2 does the same to the next backward
+ * call's key-major kernel on its first streamed tile. The consumer's bounded wait then expires
+ * and the kernel reports SKIPARSE_ERR_TIMEOUT without faulting or hanging the GPU. kind = 0
+ * clears it. A hook is consumed by one launch of the entry point it concerns. Returns
+ * SKIPARSE_OK or SKIPARSE_ERR_INVALID_ARG.
  */
 SKIPARSE_API int skiparse_debug_inject_fault(int kind);
 

@@ -147,7 +147,8 @@ def test_wait_limit_and_fault_hook(L):
     assert prev == 2_000_000_000
     assert L.skiparse_set_wait_limit_ns(0) == 123456
     assert L.skiparse_set_wait_limit_ns(0) == 2_000_000_000
-    assert L.skiparse_debug_inject_fault(2) == 1
+    assert L.skiparse_debug_inject_fault(3) == 1
+    assert L.skiparse_debug_inject_fault(2) == 0  # the backward's hook
     assert L.skiparse_debug_inject_fault(0) == 0
 
 
