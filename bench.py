@@ -360,11 +360,29 @@ def run_ours(args):
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the end-to-end timing")
+        # the transfer floor of the same bytes: plain pinned copies host -> device of q, k, v and
+        # device -> host of the output, each direction timed alone (the two directions of the
+        # link run concurrently in the pipelined call, so its floor is the slower of the two)
+        scratch = torch.empty_like(qd)
+        c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        c0.record(stream)
+        for t_h in (qh, kh, vh):
+            scratch.copy_(t_h, non_blocking=True)
+        c1.record(stream)
+        oh.copy_(out, non_blocking=True)
+        c2.record(stream)
+        torch.cuda.synchronize(dev)
+        h2d_ms, d2h_ms = c0.elapsed_time(c1), c1.elapsed_time(c2)
+        del scratch
         e2e = {"value": round(aggregate_tflops(fl, args.e2e_steps, world, e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2,
                "ms_per_step": round(e_ms / args.e2e_steps, 3), "steps": args.e2e_steps,
                "path": "skiparse2d_attn_fwd_host (C ABI, pinned host buffers, copies overlapped per head group)",
-               "heads_per_group": hg}
+               "heads_per_group": hg,
+               "copy_only_ms": {"h2d": round(h2d_ms, 3), "d2h": round(d2h_ms, 3),
+                                "h2d_gbs": round(3 * q.numel() * 2 / (h2d_ms / 1e3) / 1e9, 1),
+                                "d2h_gbs": round(q.numel() * 2 / (d2h_ms / 1e3) / 1e9, 1)},
+               "frac_of_transfer_floor": round(max(h2d_ms, d2h_ms) / (e_ms / args.e2e_steps), 4)}
         del ws, qh, kh, vh, oh
 
     # P = 1 dense attention at the same shape on the same kernel: ms/layer and sparse speedup
