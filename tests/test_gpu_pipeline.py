@@ -56,3 +56,32 @@ def test_fused_equals_rearrange_dense_unrearrange(w, mode):
     explicit = _pipeline(fps, q, k, v, w.P, mode)
     assert fps.get_device_status() == 0
     assert torch.equal(fused.view(torch.int16), explicit.view(torch.int16))
+
+
+SHAPES_1D = [
+    synth.custom(1, 3, 4, 16, 2, 64, 2, "1d_p2"),        # frame of 64 = 4 * 2^4 tokens, n = 48
+    synth.custom(1, 2, 9, 9, 1, 128, 3, "1d_p3"),        # frame of 81 = 3^4 tokens, n = 18
+    synth.custom(2, 2, 16, 16, 2, 32, 4, "1d_p4_b2"),    # frame of 256 = 4^4 tokens, n = 32
+    synth.WORKLOADS["720p"],                             # 3600 = 225 * 2^4 per frame: no padding
+]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("w", SHAPES_1D, ids=lambda w: w.name)
+def test_fused_1d_equals_rearrange_dense_unrearrange(w, mode):
+    """The same equivalence for Skiparse-1D on frames whose H*W needs no padding (a multiple
+    of P^4): skiparse1d_rearrange, dense attention per subsequence, skiparse1d_unrearrange."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import fixed_pattern_sparse_b200 as fps
+    assert fps.padded_length_1d(w.H * w.W, w.P) == w.H * w.W
+    q, k, v = (t.cuda() for t in synth.qkv(w))
+    fused = fps.skiparse1d_attn_fwd(q, k, v, w.P, mode)
+    B, T, H, W, heads, d = q.shape
+    ys = [fps.skiparse1d_rearrange(x, w.P, mode) for x in (q, k, v)]
+    n = ys[0].shape[1]
+    grid = [y.view(B * w.P * w.P, 1, 1, n, heads, d) for y in ys]
+    o = fps.skiparse2d_attn_fwd(*grid, 1, 0)
+    explicit = fps.skiparse1d_unrearrange(o.view(B * w.P * w.P, n, heads, d), q.shape, w.P, mode)
+    assert fps.get_device_status() == 0
+    assert torch.equal(fused.view(torch.int16), explicit.view(torch.int16))
