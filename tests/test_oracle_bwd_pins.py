@@ -16,7 +16,8 @@ from oracle import brute
 TOK, GRP = oracle.TOKEN_WISE, oracle.GROUP_WISE
 
 CASES = [synth.WORKLOADS["tiny"], synth.WORKLOADS["anyres"], synth.custom(2, 2, 5, 7, 2, 8, 3),
-         synth.custom(1, 1, 3, 17, 1, 4, 4), synth.custom(1, 2, 6, 6, 2, 16, 1)]
+         synth.custom(1, 1, 3, 17, 1, 4, 4), synth.custom(1, 2, 6, 6, 2, 16, 1),
+         synth.custom(1, 1, 26, 31, 1, 8, 5), synth.custom(1, 1, 9, 11, 1, 4, 8)]
 
 
 def grads_by_autograd(q, k, v, dout, P, mode):
