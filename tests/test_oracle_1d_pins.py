@@ -91,7 +91,8 @@ def test_720p_latent_needs_no_padding_and_480p_does():
 # ------------------------------------------------------------------------------- rearrange
 
 @pytest.mark.parametrize("B,T,H,W,P", [(1, 1, 4, 4, 2), (2, 3, 4, 8, 2), (1, 2, 5, 7, 2),
-                                       (1, 2, 9, 9, 3), (2, 2, 3, 5, 1)])
+                                       (1, 2, 9, 9, 3), (2, 2, 3, 5, 1), (1, 2, 13, 17, 5),
+                                       (1, 1, 30, 70, 8)])
 def test_token_wise_is_strided_slicing(B, T, H, W, P):
     """A 1D token skip with ratio k: subsequence c is x[c::k] of each (padded) frame."""
     k = P * P
@@ -106,7 +107,8 @@ def test_token_wise_is_strided_slicing(B, T, H, W, P):
 
 
 @pytest.mark.parametrize("B,T,H,W,P", [(1, 1, 4, 4, 2), (2, 2, 4, 8, 2), (1, 2, 5, 7, 2),
-                                       (1, 1, 9, 9, 3), (1, 2, 2, 3, 1)])
+                                       (1, 1, 9, 9, 3), (1, 2, 2, 3, 1), (1, 2, 13, 17, 5),
+                                       (1, 1, 30, 70, 8)])
 def test_group_wise_is_group_reshape(B, T, H, W, P):
     """A 1D group skip with ratio k: cut each padded frame into runs of k consecutive tokens;
     run m goes to subsequence m mod k, runs kept whole and in order -- a reshape of the frame to
@@ -163,7 +165,8 @@ def test_p1_is_dense_attention(shape):
 
 @pytest.mark.parametrize("mode", [TOK, GRP])
 @pytest.mark.parametrize("shape,P", [((1, 2, 4, 4, 2, 8), 2), ((2, 2, 3, 7, 1, 16), 2),
-                                     ((1, 1, 9, 10, 1, 8), 3), ((1, 2, 1, 3, 2, 8), 2)])
+                                     ((1, 1, 9, 10, 1, 8), 3), ((1, 2, 1, 3, 2, 8), 2),
+                                     ((1, 1, 13, 17, 1, 8), 5), ((1, 1, 30, 70, 1, 4), 8)])
 def test_forward_matches_brute_force_mask(mode, shape, P):
     q, k, v = (synth.randn_bf16(shape, seed=s) for s in (21, 22, 23))
     got = oracle.attn_fwd(q, k, v, P, mode, dims=1)
