@@ -44,46 +44,51 @@ _LIB = None
 def lib():
     global _LIB
     if _LIB is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        c_int, c_ll, vp = ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p
-        L.oracle_padded_extent.argtypes = [c_int, c_int]
-        L.oracle_padded_extent.restype = c_int
-        L.oracle_axis_map.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_int), ctypes.POINTER(c_int)]
-        L.oracle_axis_map.restype = c_int
-        L.oracle_subseq_len.argtypes = [c_int, c_int, c_int, c_int]
-        L.oracle_subseq_len.restype = c_ll
-        shape8 = [c_int] * 8  # B, T, H, W, heads, d, P, mode
-        L.oracle_rearrange.argtypes = [vp, vp, vp] + shape8
-        L.oracle_rearrange.restype = c_int
-        L.oracle_unrearrange.argtypes = [vp, vp] + shape8
-        L.oracle_unrearrange.restype = c_int
-        L.oracle_switch_mode.argtypes = [vp, vp] + shape8
-        L.oracle_switch_mode.restype = c_int
-        L.oracle_unrearrange_f64.argtypes = [vp, vp] + shape8
-        L.oracle_unrearrange_f64.restype = c_int
-        L.oracle_masked_attention.argtypes = [vp, vp, vp, vp, vp, c_ll, c_ll, c_int, c_int, c_int]
-        L.oracle_masked_attention.restype = c_int
-        L.oracle_attn_fwd.argtypes = [vp, vp, vp, vp] + shape8 + [c_int]
-        L.oracle_attn_fwd.restype = c_int
-        L.oracle_attn_fwd_rows.argtypes = [vp, vp, vp, vp, c_ll, vp] + shape8 + [c_int]
-        L.oracle_attn_fwd_rows.restype = c_int
-        L.oracle_attn_bwd.argtypes = [vp] * 8 + shape8 + [c_int]
-        L.oracle_attn_bwd.restype = c_int
-        L.oracle_attn_bwd_rows.argtypes = [vp, vp, vp, vp, vp, c_ll, vp, vp, vp] + shape8 + [c_int]
-        L.oracle_attn_bwd_rows.restype = c_int
-        L.oracle1d_padded_length.argtypes = [c_int, c_int]
-        L.oracle1d_padded_length.restype = c_int
-        L.oracle1d_index_map.argtypes = L.oracle_axis_map.argtypes
-        L.oracle1d_index_map.restype = c_int
-        L.oracle1d_subseq_len.argtypes = L.oracle_subseq_len.argtypes
-        L.oracle1d_subseq_len.restype = c_ll
-        for name in ("rearrange", "unrearrange", "switch_mode", "unrearrange_f64", "attn_fwd",
-                     "attn_fwd_rows", "attn_bwd", "attn_bwd_rows"):
-            f1, f2 = getattr(L, "oracle1d_" + name), getattr(L, "oracle_" + name)
-            f1.argtypes, f1.restype = f2.argtypes, f2.restype
-        _LIB = L
+        _LIB = load(_build.build())
     return _LIB
+
+
+def load(path: str):
+    """A ctypes handle on an oracle library at `path`, with every function's signature bound
+    (lib() is the normal build; the oracle's mutation tests load planted-mistake builds)."""
+    L = ctypes.CDLL(path)
+    c_int, c_ll, vp = ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p
+    L.oracle_padded_extent.argtypes = [c_int, c_int]
+    L.oracle_padded_extent.restype = c_int
+    L.oracle_axis_map.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_int), ctypes.POINTER(c_int)]
+    L.oracle_axis_map.restype = c_int
+    L.oracle_subseq_len.argtypes = [c_int, c_int, c_int, c_int]
+    L.oracle_subseq_len.restype = c_ll
+    shape8 = [c_int] * 8  # B, T, H, W, heads, d, P, mode
+    L.oracle_rearrange.argtypes = [vp, vp, vp] + shape8
+    L.oracle_rearrange.restype = c_int
+    L.oracle_unrearrange.argtypes = [vp, vp] + shape8
+    L.oracle_unrearrange.restype = c_int
+    L.oracle_switch_mode.argtypes = [vp, vp] + shape8
+    L.oracle_switch_mode.restype = c_int
+    L.oracle_unrearrange_f64.argtypes = [vp, vp] + shape8
+    L.oracle_unrearrange_f64.restype = c_int
+    L.oracle_masked_attention.argtypes = [vp, vp, vp, vp, vp, c_ll, c_ll, c_int, c_int, c_int]
+    L.oracle_masked_attention.restype = c_int
+    L.oracle_attn_fwd.argtypes = [vp, vp, vp, vp] + shape8 + [c_int]
+    L.oracle_attn_fwd.restype = c_int
+    L.oracle_attn_fwd_rows.argtypes = [vp, vp, vp, vp, c_ll, vp] + shape8 + [c_int]
+    L.oracle_attn_fwd_rows.restype = c_int
+    L.oracle_attn_bwd.argtypes = [vp] * 8 + shape8 + [c_int]
+    L.oracle_attn_bwd.restype = c_int
+    L.oracle_attn_bwd_rows.argtypes = [vp, vp, vp, vp, vp, c_ll, vp, vp, vp] + shape8 + [c_int]
+    L.oracle_attn_bwd_rows.restype = c_int
+    L.oracle1d_padded_length.argtypes = [c_int, c_int]
+    L.oracle1d_padded_length.restype = c_int
+    L.oracle1d_index_map.argtypes = L.oracle_axis_map.argtypes
+    L.oracle1d_index_map.restype = c_int
+    L.oracle1d_subseq_len.argtypes = L.oracle_subseq_len.argtypes
+    L.oracle1d_subseq_len.restype = c_ll
+    for name in ("rearrange", "unrearrange", "switch_mode", "unrearrange_f64", "attn_fwd",
+                 "attn_fwd_rows", "attn_bwd", "attn_bwd_rows"):
+        f1, f2 = getattr(L, "oracle1d_" + name), getattr(L, "oracle_" + name)
+        f1.argtypes, f1.restype = f2.argtypes, f2.restype
+    return L
 
 
 def default_threads() -> int:

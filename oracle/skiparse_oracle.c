@@ -27,6 +27,21 @@
  */
 #include "skiparse_oracle.h"
 
+/* Mutation hooks for the oracle's own tests (tests/test_oracle_mutants.py). A build with
+ * ORACLE_MUTANT = k (1..8) plants plausible mistake k, one at a time, so that the test can
+ * check that the pins catch every one of them; the normal build (0) plants none:
+ *   1 group-wise sub-grid position x div P (blocks not kept together)
+ *   2 group-wise class (x div P^2) mod P
+ *   3 softmax scale 1 instead of 1/sqrt(d)
+ *   4 exponent sign flipped, exp(m - s)
+ *   5 padding to a multiple of P instead of P^2
+ *   6 pad keys not masked (they take part in the softmax with zero vectors)
+ *   7 Skiparse-1D frame flattened column-major (x = w*H + h instead of h*W + w)
+ *   8 backward dS = P * dP (the D term dropped)                                          */
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
 #include <math.h>
 #include <pthread.h>
 #include <stdlib.h>
@@ -49,7 +64,7 @@ static int check_shape(int B, int T, int H, int W, int heads, int d, int P, int 
  * the nearest larger multiple. */
 int oracle_padded_extent(int X, int P) {
     if (X < 1 || P < 1) return -1;
-    int q = P * P;
+    int q = ORACLE_MUTANT == 5 ? P : P * P;
     return ((X + q - 1) / q) * q;
 }
 
@@ -65,8 +80,8 @@ int oracle_axis_map(int x, int P, int mode, int* cls, int* sub) {
         *cls = x % P;
         *sub = x / P;
     } else if (mode == ORACLE_GROUP_WISE) {
-        *cls = (x / P) % P;
-        *sub = (x / (P * P)) * P + (x % P);
+        *cls = ORACLE_MUTANT == 2 ? (x / (P * P)) % P : (x / P) % P;
+        *sub = ORACLE_MUTANT == 1 ? x / P : (x / (P * P)) * P + (x % P);
     } else {
         return -1;
     }
@@ -139,7 +154,8 @@ static int pattern_init(pattern* pt, int dims, int B, int T, int H, int W, int h
 
 /* Slot of padded position f of frame t of batch element b: subsequence *seq, position *pos.
  * Returns 1 for a real token (then *tok is its index ((b*T + t)*H + h)*W + w in the original
- * layout) and 0 for a pad slot. Skiparse-2D: f = h*Wp + w, class (ci, cj) from the two axis
+ * layout), 0 for a pad slot, and -1 if the slot falls outside the rearranged tensor (never
+ * for this oracle; it keeps the builds with a planted mistake from writing out of bounds). Skiparse-2D: f = h*Wp + w, class (ci, cj) from the two axis
  * maps, subsequence b*P^2 + ci*P + cj, position (t, r, s) in raster order. Skiparse-1D:
  * f = x = h*W + w, class c from the flattened-index map, subsequence b*P^2 + c, position
  * t*(F/P^2) + the position inside the class. */
@@ -153,6 +169,7 @@ static int pattern_slot(const pattern* pt, int b, int t, long long f, long long*
         oracle_axis_map(w, pt->P, pt->mode, &cj, &s);
         *seq = (long long)b * q2 + ci * pt->P + cj;
         *pos = ((long long)t * pt->R + r) * pt->S + s;
+        if (*seq < 0 || *seq >= (long long)pt->B * q2 || *pos < 0 || *pos >= pt->n) return -1;
         if (h >= pt->H || w >= pt->W) return 0;
         *tok = (((long long)b * pt->T + t) * pt->H + h) * pt->W + w;
         return 1;
@@ -161,8 +178,10 @@ static int pattern_slot(const pattern* pt, int b, int t, long long f, long long*
     oracle1d_index_map((int)f, pt->P, pt->mode, &c, &s);
     *seq = (long long)b * q2 + c;
     *pos = (long long)t * (pt->F / q2) + s;
+    if (*seq < 0 || *seq >= (long long)pt->B * q2 || *pos < 0 || *pos >= pt->n) return -1;
     if (f >= (long long)pt->H * pt->W) return 0;
-    *tok = ((long long)b * pt->T + t) * ((long long)pt->H * pt->W) + f;
+    const long long x = ORACLE_MUTANT == 7 ? (f % pt->H) * pt->W + f / pt->H : f;
+    *tok = ((long long)b * pt->T + t) * ((long long)pt->H * pt->W) + x;
     return 1;
 }
 
@@ -183,6 +202,7 @@ static void rearrange_impl(const pattern* pt, const uint16_t* x, uint16_t* y, ui
             for (long long f = 0; f < pt->F; ++f) {
                 long long seq, pos, tok = 0;
                 const int real = pattern_slot(pt, b, t, f, &seq, &pos, &tok);
+                if (real < 0) continue;
                 uint16_t* dst = y + (seq * pt->n + pos) * row;
                 for (long long e = 0; e < row; ++e) dst[e] = real ? x[tok * row + e] : 0;
                 if (valid) valid[seq * pt->n + pos] = (uint8_t)real;
@@ -196,7 +216,7 @@ static void unrearrange_impl(const pattern* pt, const void* y, void* x, int elem
         for (int t = 0; t < pt->T; ++t)
             for (long long f = 0; f < pt->F; ++f) {
                 long long seq, pos, tok = 0;
-                if (!pattern_slot(pt, b, t, f, &seq, &pos, &tok)) continue;
+                if (pattern_slot(pt, b, t, f, &seq, &pos, &tok) != 1) continue;
                 memcpy((char*)x + tok * row * elem_bytes,
                        (const char*)y + (seq * pt->n + pos) * row * elem_bytes,
                        (size_t)(row * elem_bytes));
@@ -216,9 +236,9 @@ static void switch_impl(const pattern* src, const pattern* dst, const uint16_t* 
             for (long long f = 0; f < dst->F; ++f) {
                 long long dseq, dpos, sseq, spos, tok = 0;
                 const int real = pattern_slot(dst, b, t, f, &dseq, &dpos, &tok);
+                if (real < 0) continue;
                 uint16_t* out = ydst + (dseq * dst->n + dpos) * row;
-                if (real) {
-                    pattern_slot(src, b, t, f, &sseq, &spos, &tok);
+                if (real && pattern_slot(src, b, t, f, &sseq, &spos, &tok) == 1) {
                     for (long long e = 0; e < row; ++e) out[e] = ysrc[(sseq * src->n + spos) * row + e];
                 } else {
                     for (long long e = 0; e < row; ++e) out[e] = 0;
@@ -302,10 +322,10 @@ static void attend_one(const uint16_t* yq, const uint16_t* yk, const uint16_t* y
                        long long seq, long long i, int head, double* o, double* score) {
     const long long row = (long long)heads * d;
     const uint16_t* q = yq + ((seq * n + i) * heads + head) * d;
-    const double scale = 1.0 / sqrt((double)d);
+    const double scale = ORACLE_MUTANT == 3 ? 1.0 : 1.0 / sqrt((double)d);
     double m = -INFINITY;
     for (long long j = 0; j < n; ++j) {
-        if (!valid[seq * n + j]) continue;
+        if (!valid[seq * n + j] && ORACLE_MUTANT != 6) continue;
         const uint16_t* kj = yk + (seq * n + j) * row + (long long)head * d;
         double acc = 0.0;
         for (int e = 0; e < d; ++e) acc += bf16_bits_to_double(q[e]) * bf16_bits_to_double(kj[e]);
@@ -315,8 +335,8 @@ static void attend_one(const uint16_t* yq, const uint16_t* yk, const uint16_t* y
     double denom = 0.0;
     for (int e = 0; e < d; ++e) o[e] = 0.0;
     for (long long j = 0; j < n; ++j) {
-        if (!valid[seq * n + j]) continue;
-        const double p = exp(score[j] - m);
+        if (!valid[seq * n + j] && ORACLE_MUTANT != 6) continue;
+        const double p = ORACLE_MUTANT == 4 ? exp(m - score[j]) : exp(score[j] - m);
         denom += p;
         const uint16_t* vj = yv + (seq * n + j) * row + (long long)head * d;
         for (int e = 0; e < d; ++e) o[e] += p * bf16_bits_to_double(vj[e]);
@@ -495,7 +515,7 @@ static long long* request_keys(const pattern* pt, const long long* rows, long lo
         int b, t;
         long long f, seq, pos, tok;
         pattern_locate(pt, rows[i] / pt->heads, &b, &t, &f);
-        pattern_slot(pt, b, t, f, &seq, &pos, &tok);
+        if (pattern_slot(pt, b, t, f, &seq, &pos, &tok) < 0) seq = pos = 0;
         key[2 * i] = (seq * pt->heads + head) * pt->n + pos;
         key[2 * i + 1] = i;
     }
@@ -514,7 +534,7 @@ static void gather_subseq(const pattern* pt, long long seq, int head, const uint
         for (long long f = 0; f < pt->F; ++f) {
             long long s, p, tok = 0;
             const int real = pattern_slot(pt, b, t, f, &s, &p, &tok);
-            if (s != seq) continue;
+            if (real < 0 || s != seq) continue;
             valid[p] = (uint8_t)real;
             const long long srow = tok * pt->heads + head;
             for (int i = 0; i < nbuf; ++i)
@@ -667,7 +687,7 @@ static void* bwd_worker(void* arg) {
                 const uint16_t* kj = AT(jb->yk, j);
                 double dpv = 0.0;
                 for (int e = 0; e < d; ++e) dpv += bf16_bits_to_double(doi[e]) * bf16_bits_to_double(vj[e]);
-                const double ds = p[j] * (dpv - D);
+                const double ds = ORACLE_MUTANT == 8 ? p[j] * dpv : p[j] * (dpv - D);
                 double* dvj = jb->ydv + (seq * n + j) * row + (long long)head * d;
                 double* dkj = jb->ydk + (seq * n + j) * row + (long long)head * d;
                 for (int e = 0; e < d; ++e) {
