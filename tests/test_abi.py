@@ -202,3 +202,34 @@ def test_debug_build_hook_and_exports():
     assert D.skiparse_debug_shrink_bounds(-1) == 1
     assert D.skiparse_debug_shrink_bounds(0) == 0
     assert D.skiparse_status_string(6) == b"SKIPARSE_ERR_BOUNDS"
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/skiparse.h is a C header: a C99 program that includes it compiles with gcc
+    (-std=c99 -pedantic), links against libskiparse.so and calls its host-only entry points
+    (geometry and status strings; nothing that needs a GPU)."""
+    import shutil
+    import subprocess
+    from fixed_pattern_sparse_b200 import _lib
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "skiparse.h"
+int main(void) {
+    printf("%d %lld %lld %s %s\n", skiparse_padded_extent(45, 2), skiparse_subseq_len(21, 45, 80, 2),
+           skiparse_class_len(21, 45, 80, 2, SKIPARSE_GROUP_WISE, 1, 0),
+           skiparse_status_string(SKIPARSE_ERR_TIMEOUT), skiparse_status_string(SKIPARSE_ERR_BOUNDS));
+    return skiparse2d_attn_fwd(0, 0, 0, 0, 1, 1, 1, 1, 1, 32, 2, 0, 0) == SKIPARSE_ERR_INVALID_ARG ? 0 : 1;
+}
+''')
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Werror", str(src), "-I", os.path.dirname(HEADER),
+                    "-L", libdir, "-lskiparse", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    # 720p latent, P = 2: H pads 45 -> 48; n = 21 * 24 * 40; group-wise class (1, 0) holds the
+    # rows h with (h div 2) mod 2 = 1 below 45 (11 blocks of 4 rows x 2) and 40 of the 80 columns
+    assert out[0] == "48" and out[1] == str(21 * 24 * 40) and out[2] == str(21 * 22 * 40)
+    assert out[3] == "SKIPARSE_ERR_TIMEOUT" and out[4] == "SKIPARSE_ERR_BOUNDS"
