@@ -563,6 +563,8 @@ def run_ours(args):
         err = np.abs(got - want)
         cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": nth, "kind": "oracle",
                "sample": desc, "seconds": round(dt, 2),
+               # labelled extrapolation: the whole workload's real-pair FLOPs at the sample's rate
+               "extrapolated_seconds_per_call": round(flops_real(w, modes[0]) / (val * 1e12), 1),
                "parity": {"rows": int(len(orows)), "max_abs_err": float(err.max()),
                           "mean_abs_err": float(err.mean()),
                           "ok": bool(np.isfinite(got).all() and err.max() <= 1e-2 and err.mean() <= 1e-3),
