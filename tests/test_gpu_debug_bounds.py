@@ -27,7 +27,11 @@ SHAPES = [synth.WORKLOADS["tiny"], synth.WORKLOADS["anyres"],
 def libs():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    import os
     from fixed_pattern_sparse_b200 import _lib
+    from fixed_pattern_sparse_b200 import build as libbuild
+    if not os.path.exists(_lib.DEBUG_LIB_PATH):  # a checkout where only the release build was made
+        libbuild.build(debug=True)
     return _lib.lib(), _lib.debug_lib()
 
 
