@@ -188,11 +188,12 @@ def test_host_entry_rejects_bad_arguments_synchronously(L):
     assert L.skiparse1d_attn_fwd_host(*args, 2, FAKE + 4 * big, need - 1, None) == 1
 
 
-def test_debug_build_hook_and_exports():
+def test_debug_build_hook_and_exports(L):
     """The bounds-checking debug build exports the same C ABI; only it accepts the hook that
     declares the next launch's bounds smaller (the release build has no checks)."""
     from fixed_pattern_sparse_b200 import _lib
-    R = _lib.lib()
+    libbuild.build(debug=True)  # no-op when up to date
+    R = L
     assert R.skiparse_debug_shrink_bounds(3) == 2  # SKIPARSE_ERR_UNSUPPORTED
     assert b"debug" not in R.skiparse_version()
     D = _lib.debug_lib()
@@ -204,7 +205,7 @@ def test_debug_build_hook_and_exports():
     assert D.skiparse_status_string(6) == b"SKIPARSE_ERR_BOUNDS"
 
 
-def test_header_is_plain_c_and_links(tmp_path):
+def test_header_is_plain_c_and_links(L, tmp_path):
     """include/skiparse.h is a C header: a C99 program that includes it compiles with gcc
     (-std=c99 -pedantic), links against libskiparse.so and calls its host-only entry points
     (geometry and status strings; nothing that needs a GPU)."""
