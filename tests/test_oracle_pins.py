@@ -186,7 +186,7 @@ def test_unrearrange_inverts_rearrange(B, T, H, W, heads, d, P, mode):
     assert np.array_equal(y2, y)
 
 
-@pytest.mark.parametrize("P", [1, 2, 3])
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 5])
 @pytest.mark.parametrize("mode", [TOK, GRP])
 def test_local_equivalence(P, mode):
     """核心方法: rearranging the whole sequence equals rearranging each minimal repeating
@@ -220,7 +220,8 @@ def class_membership(H, W, P, mode):
     return cls
 
 
-@pytest.mark.parametrize("P,H,W", [(2, 8, 8), (2, 12, 16), (3, 9, 18), (2, 5, 7)])
+@pytest.mark.parametrize("P,H,W", [(2, 8, 8), (2, 12, 16), (3, 9, 18), (2, 5, 7), (4, 16, 32),
+                                   (5, 25, 25)])
 def test_two_hop_interaction(P, H, W):
     """核心方法: with the two modes alternating, any two tokens interact within at most
     two attention operations (token-wise then group-wise, and the other way round)."""
