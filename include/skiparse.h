@@ -22,7 +22,10 @@
  *     bottom/right of each frame.
  *   - Softmax scale is 1/sqrt(d); no causal mask, no dropout, no bias.
  *   - Ownership: the caller allocates and owns every buffer. The library allocates no device
- *     memory per call; its only device state is one status word per device.
+ *     memory per call. Its device state: one status word per device, and the fixed workspace
+ *     of skiparse2d_attn_bwd_noalloc (a static 16 MiB array on every device that loads the
+ *     library); the host-buffer entry points also create three streams and a few events per
+ *     device on their first call there.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
  *     Argument errors are reported synchronously, before any launch, and nothing is launched.
  *     No function throws across the ABI.
