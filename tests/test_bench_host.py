@@ -1,0 +1,36 @@
+"""Host-side pieces of bench.py that define the reported numbers, checked on CPU: the FLOP
+count behind `value` (4*N*(N/P^2)*d*heads*B with N = T*Hp*Wp, the padded token count) and the
+real-pair count reported beside it (sum over classes of 4*n_c^2*d*heads*B), for every
+benchmark workload of the measurement plan."""
+
+from __future__ import annotations
+
+import pytest
+
+import bench
+import skiparse_synth as synth
+
+# (workload, padded-formula FLOPs, real-pair FLOPs token-wise / group-wise), to 4 digits
+TABLE = [
+    ("tiny", 1.049e6, 1.049e6, 1.049e6),
+    ("anyres", 8.493e7, 4.516e7, 4.792e7),
+    ("480p", 1.876e12, 1.649e12, 1.656e12),
+    ("720p", 3.329e13, 2.928e13, 2.928e13),
+    ("768p", 3.671e13, 3.671e13, 3.671e13),
+    ("768p_p3", 2.370e13, 1.631e13, 1.648e13),
+    ("768p_p1", 1.468e14, 1.468e14, 1.468e14),
+]
+
+
+@pytest.mark.parametrize("name,padded,real_tok,real_grp", TABLE, ids=[t[0] for t in TABLE])
+def test_flop_counts(name, padded, real_tok, real_grp):
+    w = synth.WORKLOADS[name]
+    assert bench.flops_padded(w) == pytest.approx(padded, rel=5e-4)
+    assert bench.flops_real(w, 0) == pytest.approx(real_tok, rel=5e-4)
+    assert bench.flops_real(w, 1) == pytest.approx(real_grp, rel=5e-4)
+
+
+def test_720p_formula_by_hand():
+    # N = 21 * 48 * 80 padded tokens, n = N / 4 per class, d = 128, 40 heads
+    N = 21 * 48 * 80
+    assert bench.flops_padded(synth.WORKLOADS["720p"]) == 4.0 * N * (N / 4) * 128 * 40
