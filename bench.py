@@ -42,31 +42,10 @@ import skiparse_synth as synth  # noqa: E402
 METRIC = "Skiparse-2D attn fwd TFLOP/s and % BF16 peak at 720p P=2; ms/layer vs P=1 dense"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic per launch of the attention kernel, from an ncu capture, keyed by the hash of
-# the kernel sources it was captured on (a changed kernel reports null until re-captured).
+# DRAM traffic per launch of the attention kernel (dram__bytes_read.sum + dram__bytes_write.sum,
+# one-pass ncu capture of the 720p launch), keyed by the hash of the kernel sources it was
+# captured on: a changed kernel reports null until it is captured again.
 KNOWN_TRAFFIC = {
-    # 480p capture (dram__bytes_read.sum + dram__bytes_write.sum = 384.1 MB per launch), scaled to
-    # the 720p launch by the ratio of token rows (7.692); traffic grows with q/k/v/out because the
-    # kernel reads each input once and writes the output once.
-    "2a906497c379c4ad": 2.955e9,
-    # the per-axis class-count kernel: 480p capture 302.5 + 80.1 MB per launch, x 7.692
-    "726002548e064429": 2.943e9,
-    # measured directly on the 720p launch (one-pass dram__bytes metrics): 2.33 GB read +
-    # 0.756 GB written = q, k, v read once and out written once
-    "5d623923e1bf3aa7": 3.086e9,
-    # the kernel with four row-sum chains, the same capture: 2.33 GB read + 0.757 GB written
-    "1e3835ddabab1731": 3.087e9,
-    # softmax waits made warp-uniform, the same capture: 2.33 GB read + 0.756 GB written
-    "e17da04fa61e70d2": 3.086e9,
-    # host-side attribute flags made atomics (device code unchanged), the same capture:
-    # 2.33 GB read + 0.756 GB written
-    "26bde2fce291ecaa": 3.086e9,
-    # row-bound checks added for the debug build (compiled out here), the same capture:
-    # 2.33 GB read + 0.756 GB written
-    "f28ade9892c14eb0": 3.086e9,
-    # a backward fault-hook field in the shared parameter header, the same capture:
-    # 2.33 GB read + 0.756 GB written
-    "8686c48250f57858": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
@@ -102,9 +81,22 @@ def flops_padded(w) -> float:
     return 4.0 * N * (N / (w.P * w.P)) * w.d * w.heads * w.B
 
 
+def axis_real_counts(X: int, P: int, mode: int):
+    """Real positions of each class along one frame axis of X real positions, counted one by one
+    from the class rule (summary page, 核心方法: token-wise x mod P, group-wise (x div P) mod P).
+    Padding only appends pad positions, so it never changes these counts. Written here, apart
+    from both the library and the oracle, so that neither the timed oracle arm nor the FLOP
+    counts depend on the code under test."""
+    counts = [0] * P
+    for x in range(X):
+        counts[x % P if mode == 0 else (x // P) % P] += 1
+    return counts
+
+
 def class_lens(w, mode):
-    import fixed_pattern_sparse_b200 as fps
-    return [fps.class_len(w.T, w.H, w.W, w.P, mode, ci, cj) for ci in range(w.P) for cj in range(w.P)]
+    """Real tokens of each class subsequence, class c = ci*P + cj, in class order."""
+    rh, rw = axis_real_counts(w.H, w.P, mode), axis_real_counts(w.W, w.P, mode)
+    return [w.T * rh[ci] * rw[cj] for ci in range(w.P) for cj in range(w.P)]
 
 
 def flops_real(w, mode) -> float:
@@ -212,45 +204,52 @@ def aggregate_tflops(flops_per_step: float, steps: int, world: int, max_total_ms
 
 # ------------------------------------------------------------------------ CPU oracle
 
-def oracle_sample_rows(w, mode, nrows: int, group: int = 0) -> np.ndarray:
-    """`nrows` query rows (token*heads + head) of one (class, head) group, for timing the
-    oracle: all real tokens of class `group % P^2`, head `group // P^2`."""
+def subsequence_rows(w, mode, cls: int, head: int) -> np.ndarray:
+    """Every query row (token*heads + head) of one (class, head) subsequence of batch element 0,
+    in token order, with the class rule from the oracle."""
     import oracle
-    q2 = w.P * w.P
-    c, head = group % q2, (group // q2) % w.heads
     toks = []
     for t in range(w.T):
         for h in range(w.H):
             ci, _ = oracle.axis_map(h, w.P, mode)
             for x in range(w.W):
                 cj, _ = oracle.axis_map(x, w.P, mode)
-                if ci * w.P + cj == c:
+                if ci * w.P + cj == cls:
                     toks.append((t * w.H + h) * w.W + x)
-    toks = np.array(toks, dtype=np.int64)
-    pick = np.linspace(0, len(toks) - 1, num=min(nrows, len(toks))).astype(np.int64)
-    return toks[pick] * w.heads + head
+    return np.array(toks, dtype=np.int64) * w.heads + head
 
 
-def time_oracle(w, q, k, v, mode, target_s: float, nthreads: int):
-    """Times the oracle on a bounded sample sized to about target_s seconds of CPU work.
-    Returns (TFLOP/s, seconds, description, sampled rows, the oracle's fp64 output rows)."""
+def oracle_sample_rows(w, mode, nrows: int, group: int = 0) -> np.ndarray:
+    """`nrows` query rows (token*heads + head), evenly spaced over one (class, head) subsequence,
+    for timing the oracle: class `group % P^2`, head `group // P^2`."""
+    q2 = w.P * w.P
+    rows = subsequence_rows(w, mode, group % q2, (group // q2) % w.heads)
+    pick = np.linspace(0, len(rows) - 1, num=min(nrows, len(rows))).astype(np.int64)
+    return rows[pick]
+
+
+def time_oracle_subsequences(w, q, k, v, modes, nthreads: int):
+    """Times the oracle on whole (class, head) subsequences: for each mode, every real query of
+    the last class and the last head (in padded workloads the raggedest subsequence). Returns
+    (TFLOP/s, seconds, description, {mode: (rows, fp64 output rows)}); the rows double as the
+    benchmark's own parity check of the kernel."""
     import oracle
-    n_c = max(class_lens(w, mode))
-    per_row = 4.0 * n_c * w.d
-    rows = oracle_sample_rows(w, mode, max(nthreads, 8))
-    t = time.perf_counter()
-    oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
-    dt = time.perf_counter() - t
-    nrows = int(min(max(len(rows) * target_s / max(dt, 1e-3), nthreads), 200000))
-    rows = oracle_sample_rows(w, mode, nrows)
-    t = time.perf_counter()
-    want = oracle.attn_fwd_rows(q, k, v, rows, w.P, mode, nthreads)
-    dt = time.perf_counter() - t
-    flops = per_row * len(rows)
-    desc = (f"{len(rows)} query rows of one (class, head) subsequence of the {w.name} workload "
-            f"({MODE_NAME[mode]}), each attending over its class's ~{n_c} real keys; the oracle's "
-            f"per-subsequence gather included")
-    return flops / dt / 1e12, dt, desc, rows, want
+    q2 = w.P * w.P
+    cls, head = q2 - 1, w.heads - 1
+    flops, secs, per_mode = 0.0, 0.0, {}
+    for m in modes:
+        rows = subsequence_rows(w, m, cls, head)
+        t = time.perf_counter()
+        want = oracle.attn_fwd_rows(q, k, v, rows, w.P, m, nthreads)
+        secs += time.perf_counter() - t
+        n_c = class_lens(w, m)[cls]
+        flops += 4.0 * n_c * w.d * len(rows)
+        per_mode[m] = (rows, want)
+    desc = ("; ".join(f"{MODE_NAME[m]}: all {len(per_mode[m][0])} query rows of the (class {cls}, head {head}) "
+                      f"subsequence of the {w.name} workload over its {len(per_mode[m][0])} real keys"
+                      for m in modes)
+            + "; the oracle's per-subsequence gather included")
+    return flops / secs / 1e12, secs, desc, per_mode
 
 
 MODE_NAME = synth.MODE_NAMES
@@ -555,20 +554,25 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         nth = oracle.default_threads()
-        val, dt, desc, orows, want = time_oracle(w, q, k, v, modes[0], args.cpu_seconds, nth)
+        val, dt, desc, per_mode = time_oracle_subsequences(w, q, k, v, modes, nth)
         # the same rows from the kernel (outside every timed region): the bench's own parity
-        # check against the oracle, at the tolerance of the parity tests
-        fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, modes[0], out=out)
-        got = out.reshape(-1, w.d).index_select(0, torch.from_numpy(orows).to(dev)).double().cpu().numpy()
-        err = np.abs(got - want)
+        # check against the oracle, whole subsequences in every mode, at the parity tests' tolerance
+        parity = {}
+        for m in modes:
+            orows, want = per_mode[m]
+            fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, m, out=out)
+            got = out.reshape(-1, w.d).index_select(0, torch.from_numpy(orows).to(dev)).double().cpu().numpy()
+            err = np.abs(got - want)
+            parity[MODE_NAME[m]] = {
+                "rows": int(len(orows)), "subsequence": f"class {w.P * w.P - 1}, head {w.heads - 1} (whole)",
+                "max_abs_err": float(err.max()), "mean_abs_err": float(err.mean()),
+                "ok": bool(np.isfinite(got).all() and err.max() <= 1e-2 and err.mean() <= 1e-3)}
+        parity["tolerance"] = "max <= 1e-2, mean <= 1e-3 against the fp64 oracle"
         cpu = {"value": round(val, 6), "unit": "TFLOP/s", "cores": nth, "kind": "oracle",
                "sample": desc, "seconds": round(dt, 2),
                # labelled extrapolation: the whole workload's real-pair FLOPs at the sample's rate
                "extrapolated_seconds_per_call": round(flops_real(w, modes[0]) / (val * 1e12), 1),
-               "parity": {"rows": int(len(orows)), "max_abs_err": float(err.max()),
-                          "mean_abs_err": float(err.mean()),
-                          "ok": bool(np.isfinite(got).all() and err.max() <= 1e-2 and err.mean() <= 1e-3),
-                          "tolerance": "max <= 1e-2, mean <= 1e-3 against the fp64 oracle"}}
+               "parity": parity}
 
     if rank == 0:
         real = {MODE_NAME[m]: round(flops_real(w, m) / (by_mode[MODE_NAME[m]] / 1e3) / 1e12, 1)
@@ -736,7 +740,6 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-heads-per-group", type=int, default=2)
     ap.add_argument("--dense-steps", type=int, default=3)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

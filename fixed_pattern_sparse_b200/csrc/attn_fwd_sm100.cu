@@ -23,9 +23,6 @@
 // exponentials of the second half run.
 // Softmax rescales O lazily: only when a row maximum grows by more than 2^8 (FlashAttention-4's
 // lazy rescaling); the stale maximum keeps every p <= 256, exact after the final division.
-// Options (compile-time, off by default because they measured no faster on B200): MUFU turns
-// between the two softmax warpgroups, part of the exponentials as a polynomial on the FMA pipe
-// (a FlashAttention-4 idea), a setmaxnreg split.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -38,36 +35,12 @@ namespace {
 
 constexpr int kBM = 128;   // queries per tile == TMEM lanes
 constexpr int kBN = 128;   // keys per tile
-// Register split: 12 warps; the softmax warpgroups raise their register budget with
-// setmaxnreg while the producer/MMA warpgroup lowers its own.
-#ifndef SKIPARSE_REGSPLIT
-#define SKIPARSE_REGSPLIT 0
-#endif
-// Optional softmax schedule, measured no faster on B200 and therefore off by default: MUFU
-// turns (the two softmax warpgroups take turns on the exponential unit).
-#ifndef SKIPARSE_MUFU_TURNS
-#define SKIPARSE_MUFU_TURNS 0
-#endif
-constexpr int kThreads = SKIPARSE_REGSPLIT ? 384 : 352;
-constexpr int kLaunchRegs = 168;       // 65536 / 384 rounded down to a multiple of 8
-[[maybe_unused]] constexpr int kSoftmaxRegs = 216;  // 2 x 128 x 216 + 128 x 64 <= 384 x 168
-[[maybe_unused]] constexpr int kOtherRegs = 64;
+constexpr int kThreads = 352;
 constexpr int kProdWarp0 = 8;
 constexpr int kNumProducers = 64;
 constexpr int kMmaWarp = 10;
-constexpr float kRescaleLog2 = 8.0f;
-// P is released to the tensor core in this many parts of the key tile (2 or 4).
-#ifndef SKIPARSE_P_PARTS
-#define SKIPARSE_P_PARTS 2
-#endif
-constexpr int kPParts = SKIPARSE_P_PARTS;
-static_assert(kPParts == 2 || kPParts == 4, "P parts");  // rescale O only when the max grows by more than 2^8
-// Which of the 16 column pairs of every 32-column chunk take exp2 on the FMA pipe (polynomial)
-// instead of the MUFU unit. 0: none (fastest measured: MUFU is not this kernel's limiter).
-#ifndef SKIPARSE_EMU_MASK
-#define SKIPARSE_EMU_MASK 0x0000u
-#endif
-constexpr unsigned kEmuMask = SKIPARSE_EMU_MASK;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+constexpr int kPParts = 2;            // P is released to the tensor core in two halves of the key tile
 
 template <int D>
 struct Cfg : TileGeom<D> {
@@ -94,8 +67,7 @@ struct Cfg : TileGeom<D> {
     static constexpr int B_VEMPTY = B_VFULL + VST;
     static constexpr int B_SFULL = B_VEMPTY + VST;        // 2: one per query tile
     static constexpr int B_PFULL = B_SFULL + 2;           // 2 x kPParts: (query tile, part of the key tile)
-    static constexpr int B_TURN = B_PFULL + 2 * kPParts;  // 2: MUFU turn of query tile 0 / 1
-    static constexpr int B_OFULL = B_TURN + 2;
+    static constexpr int B_OFULL = B_PFULL + 2 * kPParts;
     static constexpr int B_DRAIN = B_OFULL + 1;
     static constexpr int NBARS = B_DRAIN + 1;
     static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
@@ -150,7 +122,6 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
             for (int h = 0; h < kPParts; ++h) ptx::mbar_init(bar(C::B_PFULL + kPParts * i + h), kBM);
-            ptx::mbar_init(bar(C::B_TURN + i), kBM);
         }
         ptx::mbar_init(bar(C::B_OFULL), 1);
         ptx::mbar_init(bar(C::B_DRAIN), 1);
@@ -167,9 +138,6 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
     const uint32_t tmem = *tmem_slot;
 
     if (warp >= kProdWarp0) {
-#if SKIPARSE_REGSPLIT
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-#endif
       if (warp == kProdWarp0 || warp == kProdWarp0 + 1) {
         // ------------------------------------------------------------------ producers
         // Load order Q, K0, V0, K1, V1, ... Every thread arrives on a load's full barrier with
@@ -301,11 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
             ptx::mbar_wait(bar(C::B_DRAIN), 0, &never, lim);
         }
         __syncwarp();
-      }  // warp 11 (register-split layout only) has no role
+      }
     } else {
-#if SKIPARSE_REGSPLIT
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-#endif
         // ------------------------------------------------------------------ softmax (WG 0/1)
         const int qt = warp >> 2;                       // query tile 0 or 1
         const int row = threadIdx.x & 127;              // TMEM lane == row in the tile
@@ -313,14 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
         const uint32_t s_addr = tmem + lane_base + (qt ? C::COL_S1 : C::COL_S0);
         const uint32_t o_col = qt ? C::COL_O1 : C::COL_O0;
         const uint32_t sfull = bar(C::B_SFULL + qt);
-        // The two query tiles take turns on the MUFU unit (their exponential phases would
-        // otherwise overlap and each would run at half rate).
-        const uint32_t my_turn = bar(C::B_TURN + qt), other_turn = bar(C::B_TURN + (qt ^ 1));
         const float sl2 = p.scale_log2;
         const float thresh = kRescaleLog2 / sl2;       // in raw score units
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        if (SKIPARSE_MUFU_TURNS && qt == 1) ptx::mbar_arrive(bar(C::B_TURN + 0));  // tile 0 goes first
         for (int j = 0; j < nkv; ++j) {
             // Every wait of a softmax warp is made uniform over the warp (a lane can see the abort
             // flag while another sees the phase complete): the tcgen05.ld/st below are
@@ -368,10 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 alpha = (j == 0) ? 0.f : ptx::ex2_approx((m_run - mx) * sl2);
                 m_run = mx;
             }
-            if (SKIPARSE_MUFU_TURNS && !__all_sync(0xffffffffu, ptx::mbar_wait(my_turn, j & 1, abort, lim))) {
-                ok = false;
-                break;
-            }
             // P = 2^(S*scale*log2(e) - m), written as bf16 pairs over the first 64 columns of S.
             // Each half of the key tile is released to the tensor core as soon as it is stored,
             // so O += P V on the first half overlaps the exponentials of the second.
@@ -384,14 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                 for (int e = 0; e < 16; ++e) {
                     const float x0 = fmaf(sc[32 * g + 2 * e], sl2, neg);
                     const float x1 = fmaf(sc[32 * g + 2 * e + 1], sl2, neg);
-                    float p0, p1;
-                    if (kEmuMask != 0u && !last && (kEmuMask & (1u << e))) {
-                        p0 = ptx::exp2_poly(x0);
-                        p1 = ptx::exp2_poly(x1);
-                    } else {
-                        p0 = ptx::ex2_approx(x0);
-                        p1 = ptx::ex2_approx(x1);
-                    }
+                    const float p0 = ptx::ex2_approx(x0);
+                    const float p1 = ptx::ex2_approx(x1);
                     if (e & 1) {
                         sum2 += p0;
                         sum3 += p1;
@@ -402,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                     pk[e] = ptx::pack_bf16x2(p0, p1);
                 }
                 ptx::tmem_st16(s_addr + 16 * g, pk);
-                if (g == (kPParts == 4 ? 0 : 1) && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (g == 1 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     // Rare: a row max grew by more than 2^8. This warp rescales its rows of O_qt
                     // before releasing the first half of P, i.e. before this tile's P*V
                     // accumulates into O_qt; O_qt was completed by the previous P*V (the commit
@@ -419,13 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1) skiparse_attn_fwd_kernel(const At
                         ptx::tmem_st16(o_addr, ov);
                     }
                 }
-                if (kPParts == 4 || (g & 1)) {
+                if (g & 1) {
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
-                    ptx::mbar_arrive(bar(C::B_PFULL + kPParts * qt + (kPParts == 4 ? g : g >> 1)));
+                    ptx::mbar_arrive(bar(C::B_PFULL + kPParts * qt + (g >> 1)));
                 }
             }
-            if (SKIPARSE_MUFU_TURNS) ptx::mbar_arrive(other_turn);
             l_run = l_run * alpha + ((sum0 + sum1) + (sum2 + sum3));
         }
         if (ok && __all_sync(0xffffffffu, ptx::mbar_wait(bar(C::B_OFULL), 0, abort, lim))) {
@@ -482,14 +432,6 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
         e = cudaFuncSetAttribute(skiparse_attn_fwd_kernel<D>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return static_cast<int>(e);
-        if (SKIPARSE_REGSPLIT) {
-            // setmaxnreg.inc waits for registers that the block released; the split above is
-            // only safe if the block is launched with exactly kLaunchRegs per thread.
-            cudaFuncAttributes fa;
-            e = cudaFuncGetAttributes(&fa, skiparse_attn_fwd_kernel<D>);
-            if (e != cudaSuccess) return static_cast<int>(e);
-            if (fa.numRegs != kLaunchRegs) return static_cast<int>(cudaErrorInvalidConfiguration);
-        }
         attr_done_dev[dev].store(1, std::memory_order_release);
     }
     int n_max = 0;
@@ -503,33 +445,20 @@ int launch_d(const AttnParams& p, const Geometry& g, cudaStream_t stream) {
     return static_cast<int>(cudaGetLastError());
 }
 
-// Diagnostic: y = 2^x by the MUFU instruction (method 0) or the FMA-pipe polynomial (method 1)
-// exactly as the softmax evaluates them, so their error can be tested against fp64.
-__global__ void skiparse_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n,
-                                     int method) {
-    const long long i = 2 * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
-    if (i >= n) return;
-    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
-    float y0, y1;
-    if (method == 1) {
-        y0 = ptx::exp2_poly(x0);
-        y1 = ptx::exp2_poly(x1);
-    } else {
-        y0 = ptx::ex2_approx(x0);
-        y1 = ptx::ex2_approx(x1);
-    }
-    y[i] = y0;
-    if (i + 1 < n) y[i + 1] = y1;
+// Diagnostic: y = 2^x by the MUFU instruction exactly as the softmax evaluates it, so its
+// error can be tested against fp64.
+__global__ void skiparse_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = ptx::ex2_approx(x[i]);
 }
 
 }  // namespace
 
-int launch_exp2(const float* x, float* y, long long n, int method, void* stream) {
+int launch_exp2(const float* x, float* y, long long n, void* stream) {
     if (n <= 0) return static_cast<int>(cudaSuccess);
-    const long long pairs = (n + 1) / 2;
     const int threads = 256;
-    const long long blocks = (pairs + threads - 1) / threads;
-    skiparse_exp2_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, method);
+    const long long blocks = (n + threads - 1) / threads;
+    skiparse_exp2_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
     return static_cast<int>(cudaGetLastError());
 }
 

@@ -10,8 +10,6 @@
 // the kernels of skiparse2d_attn_bwd.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/skiparse.h"
 
 namespace {
@@ -21,30 +19,17 @@ constexpr long long kNoAllocMaxRows = 1LL << 22;
 
 static __device__ __align__(256) float g_bwd_workspace[kNoAllocMaxRows];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-float* g_workspace_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the workspace on the current device. In host code the array's name is only
-// a stand-in for the symbol, never a device address, so the address is asked for once per
-// device (with that device current) and cached.
-int workspace_on_current_device(float** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
+// Device address of the workspace in the current device's context. In host code the array's
+// name is only a stand-in for the symbol, never a device address, so the address is asked for
+// on every call: a cached address could belong to a context that cudaDeviceReset has since
+// destroyed, or to another context the caller made current. The lookup allocates nothing.
+int workspace_in_current_context(float** out) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_workspace) != cudaSuccess || !ptr) {
         cudaGetLastError();
         return SKIPARSE_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) return SKIPARSE_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_workspace_ptr[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_bwd_workspace) != cudaSuccess || !ptr) {
-            cudaGetLastError();
-            return SKIPARSE_ERR_CUDA;
-        }
-        g_workspace_ptr[dev] = static_cast<float*>(ptr);
-    }
-    *out = g_workspace_ptr[dev];
+    *out = static_cast<float*>(ptr);
     return SKIPARSE_OK;
 }
 
@@ -55,12 +40,16 @@ extern "C" int skiparse2d_attn_bwd_noalloc(const void* q, const void* k, const v
                                            void* dq, void* dk, void* dv, int B, int T, int H,
                                            int W, int heads, int d, int P, int mode,
                                            skiparse_stream_t stream) {
-    if (B > 0 && T > 0 && H > 0 && W > 0 && heads > 0) {
-        const long long rows = static_cast<long long>(B) * T * H * W * heads;
-        if (rows > kNoAllocMaxRows) return SKIPARSE_ERR_UNSUPPORTED;  // workspace too small
-    }
+    // Argument errors first, before any CUDA call, in the order and with the codes of
+    // skiparse2d_attn_bwd (which checks the rest -- alignment, overlaps -- before it launches).
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return SKIPARSE_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || P < 1) return SKIPARSE_ERR_INVALID_ARG;
+    if (mode != SKIPARSE_TOKEN_WISE && mode != SKIPARSE_GROUP_WISE) return SKIPARSE_ERR_INVALID_ARG;
+    if (P > 8 || (d != 32 && d != 64 && d != 128)) return SKIPARSE_ERR_UNSUPPORTED;
+    const long long rows = static_cast<long long>(B) * T * H * W * heads;
+    if (rows > kNoAllocMaxRows) return SKIPARSE_ERR_UNSUPPORTED;  // workspace too small
     float* workspace = nullptr;
-    const int st = workspace_on_current_device(&workspace);
+    const int st = workspace_in_current_context(&workspace);
     if (st != SKIPARSE_OK) return st;
     // The workspace is written in full by the first of the backward's launches before anything
     // reads it, so the previous call's contents never matter and nothing needs clearing.

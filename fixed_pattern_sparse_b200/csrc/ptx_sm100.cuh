@@ -1,13 +1,12 @@
 // ptx_sm100.cuh -- hand-written inline-PTX wrappers for sm_100a used by the Skiparse kernels:
-// mbarriers with bounded waits, TMA (tile::gather4) loads, and the 5th-generation tensor-core
-// path (tcgen05: TMEM allocation, MMA, commit, TMEM loads/stores, fences).
+// mbarriers with bounded waits and the 5th-generation tensor-core path (tcgen05: TMEM
+// allocation, MMA, commit, TMEM loads/stores, fences).
 //
 // Descriptor encodings follow the PTX ISA's tcgen05 "shared memory descriptor" and
 // "instruction descriptor" tables (kind::f16, bf16 inputs, fp32 accumulate).
 #pragma once
 
 #include <cstdint>
-#include <cuda.h>
 
 namespace skiparse {
 namespace ptx {
@@ -20,12 +19,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
-}
-
-__device__ __forceinline__ uint32_t lane_id() {
-    uint32_t l;
-    asm volatile("mov.u32 %0, %%laneid;" : "=r"(l));
-    return l;
 }
 
 // ------------------------------------------------------------------------------ mbarrier
@@ -42,27 +35,8 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-// A thread that finds the phase incomplete may be suspended (not spinning) until the phase
-// completes or about `SKIPARSE_WAIT_HINT_NS` nanoseconds pass (0: the hardware default).
-#ifndef SKIPARSE_WAIT_HINT_NS
-#define SKIPARSE_WAIT_HINT_NS 0
-#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-#if SKIPARSE_WAIT_HINT_NS > 0
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(static_cast<uint32_t>(SKIPARSE_WAIT_HINT_NS))
-        : "memory");
-#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -70,50 +44,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
-#endif
     return ok != 0;
 }
 
 // Waits for the phase with the given parity to complete. Bounded: gives up (returns false)
 // when *abort becomes non-zero or after limit_ns nanoseconds, so that a lost arrival can
 // never hang the GPU.
-// A waiting warp backs off with nanosleep so that it does not take issue slots from the warps
-// doing the work on the same SM sub-partition (0 disables the back-off).
-#ifndef SKIPARSE_WAIT_SLEEP_NS
-#define SKIPARSE_WAIT_SLEEP_NS 0
-#endif
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (SKIPARSE_WAIT_SLEEP_NS > 0) __nanosleep(SKIPARSE_WAIT_SLEEP_NS);
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0u) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) return false;
         }
     }
-}
-
-// -------------------------------------------------------------------------------- TMA
-
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// Loads 4 arbitrary rows (row0..row3) x one box width of columns starting at `col` of a 2-D
-// tensor map whose box is one row high, into 4 consecutive box rows at `dst` (swizzled as
-// the map says), completing `bytes` transactions on `bar`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t col, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(bar)
-        : "memory");
 }
 
 // --------------------------------------------------------------------------- tcgen05
@@ -181,8 +128,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 
 #define SKP_R8(i) "=r"(v[i + 0]), "=r"(v[i + 1]), "=r"(v[i + 2]), "=r"(v[i + 3]), \
                   "=r"(v[i + 4]), "=r"(v[i + 5]), "=r"(v[i + 6]), "=r"(v[i + 7])
-#define SKP_W8(i) "r"(v[i + 0]), "r"(v[i + 1]), "r"(v[i + 2]), "r"(v[i + 3]), \
-                  "r"(v[i + 4]), "r"(v[i + 5]), "r"(v[i + 6]), "r"(v[i + 7])
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -205,17 +150,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         : "memory");
 }
 
-// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-            taddr),
-        SKP_W8(0), SKP_W8(8), SKP_W8(16), SKP_W8(24)
-        : "memory");
-}
-
 #define SKP_W16 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), \
                 "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), \
                 "r"(v[14]), "r"(v[15])
@@ -231,7 +165,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 
 #undef SKP_W16
 #undef SKP_R8
-#undef SKP_W8
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading- and stride-dimension
 // byte offsets (all in 16-byte units), descriptor version 1, and the swizzle layout
@@ -270,46 +203,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// ---------------------------------------------------------------- packed fp32 (sm_100)
-
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// 2^x for a pair of floats on the FMA pipe instead of the MUFU unit: x = n + f with n the
-// nearest integer (added to the exponent field) and f in [-1/2, 1/2], where 2^f is a degree-3
-// polynomial. Its coefficients were fitted here with the Remez exchange algorithm (minimax
-// relative error) and give max relative error 7.5e-5 in fp32 Horner form, 26x below half an
-// ulp of bf16, the precision P is kept in. x is clamped at -125 so the exponent field cannot
-// underflow (2^-125 ~ 2.4e-38 stands in for smaller results).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.f);                             // keeps n + 127 inside the exponent field
-    const float t = x + 12582912.f;                   // 1.5 * 2^23: round(x) in the low bits
-    const float f = x - (t - 12582912.f);             // f in [-1/2, 1/2]
-    float p = fmaf(0.0551716685f, f, 0.242611125f);
-    p = fmaf(p, f, 0.693260968f);
-    p = fmaf(p, f, 0.999928057f);
-    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));  // n << 23 added
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -202,9 +202,9 @@ int skiparse_debug_shrink_bounds(long long rows) {
 
 int skiparse_debug_exp2(const float* x, float* y, long long n, int method,
                         skiparse_stream_t stream) {
-    if (n < 0 || (n > 0 && (!x || !y)) || (method != 0 && method != 1)) return SKIPARSE_ERR_INVALID_ARG;
+    if (n < 0 || (n > 0 && (!x || !y)) || method != 0) return SKIPARSE_ERR_INVALID_ARG;
     if (n >= (1ll << 40)) return SKIPARSE_ERR_UNSUPPORTED;
-    const int e = skiparse::launch_exp2(x, y, n, method, stream);
+    const int e = skiparse::launch_exp2(x, y, n, stream);
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 

@@ -118,9 +118,12 @@ SKIPARSE_API int skiparse2d_attn_bwd(const void* q, const void* k, const void* v
  *   - B*T*H*W*heads must be at most 4,194,304; larger problems get SKIPARSE_ERR_UNSUPPORTED
  *     before anything is launched (use skiparse2d_attn_bwd with your own workspace instead).
  *   - Allocates nothing: no cudaMalloc or cudaFree, no allocating library call.
- *   - The first call on a device looks up the workspace's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make that first call
- *     before any stream capture.
+ *   - Argument errors are reported first, before any CUDA call, with the codes of
+ *     skiparse2d_attn_bwd.
+ *   - Every call looks up the workspace's device address in the current context
+ *     (cudaGetSymbolAddress, which allocates nothing), so a reset device or another current
+ *     context never sees a stale address. The first use of the library on a device loads its
+ *     kernels and this array there: make a first call on each device before any stream capture.
  *   - All calls share the one workspace per device: calls that can run at the same time on
  *     the GPU (on different streams) race on it and must be ordered by the caller. The
  *     previous call's contents never matter; nothing needs clearing between calls.
@@ -308,9 +311,8 @@ SKIPARSE_API int skiparse_debug_shrink_bounds(long long rows);
 
 /*
  * Diagnostic (no counterpart on the pages): y[i] = 2^x[i] for n fp32 device values, evaluated
- * exactly as the attention softmax does -- method 0 with the MUFU ex2.approx instruction,
- * method 1 with the FMA-pipe degree-3 polynomial that takes part of the exponentials off the
- * MUFU unit (inputs below -125 give about 2^-125). x and y are device pointers, n >= 0;
+ * exactly as the attention softmax does, with the MUFU ex2.approx instruction (method must be
+ * 0; other values are SKIPARSE_ERR_INVALID_ARG). x and y are device pointers, n >= 0;
  * asynchronous on `stream`. Returns SKIPARSE_OK, SKIPARSE_ERR_INVALID_ARG or SKIPARSE_ERR_CUDA.
  */
 SKIPARSE_API int skiparse_debug_exp2(const float* x, float* y, long long n, int method,

@@ -71,3 +71,15 @@ def sample_rows_one_class_1d(w, mode: int, count: int, cls: int = 0, head: int =
     rng = np.random.default_rng(seed)
     pick = np.unique(np.concatenate([toks[:2], toks[-2:], rng.choice(toks, size=min(count, len(toks)), replace=False)]))
     return pick.astype(np.int64) * w.heads + head
+
+
+def subsequence_rows(w, mode: int, cls: int, head: int, b: int = 0) -> np.ndarray:
+    """Every row (token*heads + head) of one whole (b, class, head) subsequence, in token order,
+    with the class rule from the brute force's own restatement."""
+    from oracle import brute
+    step = w.P * w.P
+    Hp, Wp = -(-w.H // step) * step, -(-w.W // step) * step
+    grid = brute.class_grid(Hp, Wp, w.P, mode)[: w.H, : w.W]
+    hh, ww = np.nonzero(grid == cls)
+    toks = (b * w.T * w.H * w.W + np.arange(w.T)[:, None] * w.H * w.W + (hh * w.W + ww)[None, :]).reshape(-1)
+    return np.sort(toks).astype(np.int64) * w.heads + head

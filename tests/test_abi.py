@@ -134,6 +134,21 @@ def test_attn_fwd_rejects_bad_arguments_synchronously(L, args, code):
     assert L.skiparse2d_attn_fwd(*args, None) == code
 
 
+def test_noalloc_backward_rejects_bad_arguments_before_any_cuda_call(L):
+    """The allocation-free backward checks its arguments first, with the regular backward's
+    codes, and its workspace capacity next; on this host (no GPU) any CUDA call would fail with
+    SKIPARSE_ERR_CUDA instead."""
+    f = L.skiparse2d_attn_bwd_noalloc
+    good = (1, 2, 8, 8, 2, 32, 2, 0)
+    assert f(0, *([FAKE] * 8), *good, None) == 1                       # null q
+    assert f(*([FAKE] * 8), 0, *good, None) == 1                       # null dv
+    assert f(*([FAKE] * 9), 1, 2, 8, 8, 2, 32, 2, 2, None) == 1        # bad mode
+    assert f(*([FAKE] * 9), 0, 2, 8, 8, 2, 32, 2, 0, None) == 1        # B = 0
+    assert f(*([FAKE] * 9), 1, 2, 8, 8, 2, 48, 2, 0, None) == 2        # d = 48
+    assert f(*([FAKE] * 9), 1, 2, 8, 8, 2, 32, 9, 0, None) == 2        # P = 9
+    assert f(*([FAKE] * 9), 1, 1, 1, (1 << 22) + 1, 1, 32, 2, 0, None) == 2  # beyond the workspace
+
+
 def test_rearrange_rejects_bad_arguments_synchronously(L):
     assert L.skiparse_rearrange(0, FAKE, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
     assert L.skiparse_rearrange(FAKE, FAKE + 4, 1, 2, 8, 8, 2, 32, 2, 0, None) == 3

@@ -34,3 +34,34 @@ def test_720p_formula_by_hand():
     # N = 21 * 48 * 80 padded tokens, n = N / 4 per class, d = 128, 40 heads
     N = 21 * 48 * 80
     assert bench.flops_padded(synth.WORKLOADS["720p"]) == 4.0 * N * (N / 4) * 128 * 40
+
+
+@pytest.mark.parametrize("name", ["tiny", "anyres", "480p", "720p", "768p", "768p_p3"])
+def test_class_lens_match_the_library_geometry(name):
+    """bench.py counts class sizes itself (so that its oracle arm never loads the library); the
+    counts must still agree with the library's host geometry."""
+    import fixed_pattern_sparse_b200 as fps
+    w = synth.WORKLOADS[name]
+    for mode in (0, 1):
+        want = [fps.class_len(w.T, w.H, w.W, w.P, mode, ci, cj) for ci in range(w.P) for cj in range(w.P)]
+        assert bench.class_lens(w, mode) == want
+
+
+def test_reference_arm_loads_only_the_oracle():
+    """`bench.py --impl reference` times the oracle; nothing of the product may be imported or
+    loaded on that path."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, json, bench; bench.main(['--impl', 'reference', '--workload', 'tiny', '--steps', '1', "
+            "'--warmup', '0']); mods = [m for m in sys.modules if m.startswith('fixed_pattern_sparse_b200')]; "
+            "maps = open('/proc/self/maps').read(); print(json.dumps({'mods': mods, 'lib': 'libskiparse' in maps}))")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["value"] > 0
+    check = json.loads(lines[-1])
+    assert check == {"mods": [], "lib": False}

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import skiparse_synth as synth
-from parity_helpers import check_close, gpu_rows, sample_rows
+from parity_helpers import check_close, gpu_rows, sample_rows, subsequence_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +81,30 @@ def test_attention_full_size_sampled(fps, name, mode):
     rows = sample_rows(w, 160 if w.P == 1 else 320, seed=w.family * 10 + mode)
     want = oracle.attn_fwd_rows(q, k, v, rows, w.P, mode)
     check_close(gpu_rows(out, rows), want, f"{name} mode={mode}")
+
+
+# Whole subsequences at full size: every query of one (class, head), element by element, in the
+# launch configuration the benchmark times. The last class and the last head are the raggedest in
+# padded workloads (720p: 45 rows padded to 48; 768p P = 3: 48x84 padded to 54x90); group-wise
+# classes differ from token-wise ones only through the row map, which these cover in full.
+WHOLE = [("720p", TOK, -1), ("720p", GRP, -1), ("768p_p3", TOK, -1), ("768p_p3", GRP, -1),
+         ("768p_p3", GRP, 4)]
+
+
+@pytest.mark.parametrize("name,mode,cls", WHOLE, ids=[f"{n}-{'grp' if m else 'tok'}-c{c}" for n, m, c in WHOLE])
+def test_attention_whole_subsequence(fps, name, mode, cls):
+    w = synth.WORKLOADS[name]
+    cls = cls % (w.P * w.P)
+    head = w.heads - 1
+    q, k, v = synth.qkv(w)
+    qd, kd, vd = _dev((q, k, v))
+    out = torch.full_like(qd, float("nan"))
+    fps.skiparse2d_attn_fwd(qd, kd, vd, w.P, mode, out=out)
+    assert fps.get_device_status() == 0
+    rows = subsequence_rows(w, mode, cls, head)
+    assert len(rows) > 8000
+    want = oracle.attn_fwd_rows(q, k, v, rows, w.P, mode)
+    check_close(gpu_rows(out, rows), want, f"{name} mode={mode} class={cls} head={head} ({len(rows)} rows)")
 
 
 def test_attention_is_deterministic_and_stream_ordered(fps):

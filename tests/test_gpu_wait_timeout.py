@@ -1,9 +1,11 @@
-"""Failure detection without a GPU fault: every wait in the attention kernel is bounded.
+"""Failure detection without a GPU fault: every wait in the attention kernels is bounded.
 
-The test hook makes one launch expect 16 more bytes on its first K-tile barrier than the
-TMA ever delivers, so the MMA warp's wait runs out (a flag that nothing sets). The kernel
-must then record SKIPARSE_ERR_TIMEOUT in the device status word, release its tensor
-memory and return; the context stays usable and the next launch is correct."""
+The test hook (skiparse_debug_inject_fault) makes one producer thread of the next launch skip
+its cp.async arrival on the first K-tile barrier (forward) or on the first streamed tile's
+barrier (backward, key-major kernel). That barrier then never completes -- a flag that nothing
+sets -- so the MMA warp's bounded wait runs out. The kernel must record SKIPARSE_ERR_TIMEOUT in
+the device status word, release its tensor memory and return; the context stays usable and the
+next launch is correct."""
 
 from __future__ import annotations
 
