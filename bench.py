@@ -46,6 +46,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one-pass ncu capture of the 720p launch), keyed by the hash of the kernel sources it was
 # captured on: a changed kernel reports null until it is captured again.
 KNOWN_TRAFFIC = {
+    # the forward with the unused options removed: 2.33 GB read + 0.756 GB written (q, k, v read
+    # once, out written once)
+    "82168c2466cfad85": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
@@ -267,6 +270,80 @@ class nvtx_range:
 
     def __exit__(self, *exc):
         torch.cuda.nvtx.range_pop()
+
+
+# ------------------------------------------------------------- per-config table
+
+TABLE_WORKLOADS = ("480p", "768p", "768p_p3")
+
+
+def time_calls(fn, n, stream):
+    """Mean ms per call of fn() over n calls after two untimed ones (CUDA events on `stream`)."""
+    for _ in range(2):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def time_config_table(fps, dev, stream, peaks, args):
+    """ms per call, TFLOP/s by the padded and the real-pair formulas and the fraction of the
+    measured burst bf16 peak for every (workload, mode) of the measurement plan other than the
+    headline one; the dense P = 1 call at 768p and the sparse speedups t(P=1) / t(P); the 768p
+    backward at P = 2 and P = 3. Inputs are larger than L2 except at 480p (0.26 GB of q/k/v),
+    whose calls are timed back to back."""
+    peak = float(peaks["bf16_tflops"])
+    rows = {}
+    n = args.table_steps
+    for name in TABLE_WORKLOADS:
+        w = synth.WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in synth.qkv(w))
+        out = torch.empty_like(q)
+        fl = flops_padded(w)
+        for m in (0, 1):
+            ms = time_calls(lambda: fps.skiparse2d_attn_fwd(q, k, v, w.P, m, out=out), n, stream)
+            rows[f"{name} {MODE_NAME[m]}"] = {
+                "workload": describe(w), "ms_per_call": round(ms, 3),
+                "tflops_padded": round(fl / (ms / 1e3) / 1e12, 1),
+                "tflops_real_pairs": round(flops_real(w, m) / (ms / 1e3) / 1e12, 1),
+                "frac_of_burst_peak": round(fl / (ms / 1e3) / 1e12 / peak, 4)}
+        del q, k, v, out
+    w1 = synth.WORKLOADS["768p_p1"]
+    q, k, v = (t.to(dev) for t in synth.qkv(w1))
+    out = torch.empty_like(q)
+    ms1 = time_calls(lambda: fps.skiparse2d_attn_fwd(q, k, v, 1, 0, out=out), max(2, n // 2), stream)
+    fl1 = flops_padded(w1)
+    rows["768p_p1 dense"] = {"workload": describe(w1), "ms_per_call": round(ms1, 3),
+                             "tflops_padded": round(fl1 / (ms1 / 1e3) / 1e12, 1),
+                             "frac_of_burst_peak": round(fl1 / (ms1 / 1e3) / 1e12 / peak, 4)}
+    speedup = {f"t(P=1)/t({name} {MODE_NAME[m]})": round(ms1 / rows[f"{name} {MODE_NAME[m]}"]["ms_per_call"], 3)
+               for name in ("768p", "768p_p3") for m in (0, 1)}
+    # backward at 768p: the inputs above (same latent), P = 2 and P = 3
+    bwd = {}
+    if not args.no_backward:
+        g = synth.randn_bf16(w1.shape, 1000 * w1.family + 7).to(dev)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        delta = torch.empty(q.shape[:5], dtype=torch.float32, device=dev)
+        for P in (2, 3):
+            wP = synth.custom(w1.B, w1.T, w1.H, w1.W, w1.heads, w1.d, P)
+            for m in (0, 1):
+                o, lse = fps.skiparse2d_attn_fwd_lse(q, k, v, P, m)
+                ms = time_calls(lambda: fps.skiparse2d_attn_bwd(q, k, v, o, g, lse, P, m, dq=dq, dk=dk, dv=dv,
+                                                                delta=delta), max(2, n // 2), stream)
+                bwd[f"768p P={P} {MODE_NAME[m]}"] = {"ms_per_call": round(ms, 3),
+                                                     "tflops": round(2.5 * flops_padded(wP) / (ms / 1e3) / 1e12, 1)}
+                del o, lse
+        bwd["flop_formula"] = "2.5 x the forward's padded-formula FLOPs"
+        del g, dq, dk, dv, delta
+    del q, k, v, out
+    if fps.get_device_status() != 0:
+        raise SystemExit("device status error in the per-config timing")
+    return {"forward": rows, "sparse_speedup_768p": speedup, "backward_768p": bwd or None,
+            "steps_per_entry": n}
 
 
 # --------------------------------------------------------------------------- our arm
@@ -550,6 +627,16 @@ def run_ours(args):
         if fps.get_device_status() != 0:
             raise SystemExit("device status error in the rearrange timing")
 
+    # the measurement plan's other workloads (480p, 768p at P = 2 and P = 3, 768p P = 1 dense), each
+    # mode timed on its own, the sparse speedups against dense at 768p, and the 768p backward
+    configs = None
+    if not args.no_configs:
+        configs = time_config_table(fps, dev, stream, peaks, args)
+
+    stack = None
+    if not args.no_stack:
+        stack = time_stack(fps, w, qd, kd, vd, args.layers, args.dense_front, args.dense_back, 1, world, dev, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -601,6 +688,8 @@ def run_ours(args):
             "skiparse1d": one_d,
             "rearrange_kernels": rearr,
             "backward": bwd,
+            "configs": configs,
+            "stack": stack,
             "kernel_hash": kernel_hash(),
         }
         print(json.dumps(line), flush=True)
@@ -611,10 +700,14 @@ def run_ours(args):
 
 # ------------------------------------------------------------- hybrid stack harness
 
+STACK_RULE = "layer l's output is layer l+1's q; k and v are the same for every layer"
+
+
 def stack_schedule(layers: int, dense_front: int, dense_back: int):
     """(P, mode) per layer of a hybrid stack: dense (P=1) blocks at both ends, Skiparse-2D in
     the middle with token-wise and group-wise layers alternating (summary page 核心方法 /
-    实验结果: 4 full-attention blocks at the front and 4 at the back, the rest sparse)."""
+    实验结果: 4 full-attention blocks at the front and 4 at the back, the rest sparse).
+    P is None for the sparse layers (the workload's P)."""
     sched, k = [], 0
     for i in range(layers):
         if i < dense_front or i >= layers - dense_back:
@@ -625,6 +718,55 @@ def stack_schedule(layers: int, dense_front: int, dense_back: int):
     return sched
 
 
+def stack_pass(fps, x0, k, v, sched, bufs, keep=None):
+    """One pass of a chained attention stack: layer l attends with q = x_l (x_0 = x0) over the
+    fixed k and v, and its output is x_{l+1}. Outputs alternate between the two buffers of
+    `bufs`, so no layer's output aliases its own q. `keep` collects every layer's output (a
+    copy) when given. Returns the last layer's output."""
+    x = x0
+    for layer, (P, mode) in enumerate(sched):
+        out = bufs[layer % 2]
+        fps.skiparse2d_attn_fwd(x, k, v, P, mode, out=out)
+        if keep is not None:
+            keep.append(out.clone())
+        x = out
+    return x
+
+
+def time_stack(fps, w, q, k, v, layers, dense_front, dense_back, steps, world, dev, stream):
+    """Times the chained hybrid stack and the all-dense stack of the same depth (one pass = all
+    layers in order, each layer's launch reading the previous layer's output from HBM)."""
+    hybrid = [(w.P if p is None else p, m) for p, m in stack_schedule(layers, dense_front, dense_back)]
+    dense = [(1, 0)] * layers
+    bufs = (torch.empty_like(q), torch.empty_like(q))
+
+    def timed(sched, n):
+        stack_pass(fps, q, k, v, sched, bufs)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            stack_pass(fps, q, k, v, sched, bufs)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+
+    with nvtx_range("chained hybrid stack"):
+        h_ms = timed(hybrid, steps)
+    with nvtx_range("chained dense stack"):
+        d_ms = timed(dense, steps)
+    if fps.get_device_status() != 0:
+        raise SystemExit("device status error in the stack timing")
+    fl_h = sum(flops_padded(synth.custom(w.B, w.T, w.H, w.W, w.heads, w.d, P)) for P, _ in hybrid)
+    return {"layers": layers, "dense_front": dense_front, "dense_back": dense_back,
+            "sparse_layers": layers - dense_front - dense_back,
+            "sparse_modes": "alternating token-wise / group-wise", "chaining": STACK_RULE,
+            "ms_per_pass": round(h_ms, 2), "dense_stack_ms": round(d_ms, 2),
+            "attention_speedup": round(d_ms / h_ms, 3), "hybrid_tflops": round(fl_h / (h_ms / 1e3) / 1e12, 1),
+            "gpu_launches_per_pass": layers, "passes_timed": steps}
+
+
 def run_stack(args):
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
@@ -633,46 +775,23 @@ def run_stack(args):
     import fixed_pattern_sparse_b200 as fps
     w = synth.WORKLOADS[args.workload]
     q, k, v = (t.to(dev) for t in synth.qkv(w))
-    out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
-    hybrid = [(w.P if p is None else p, m) for p, m in stack_schedule(args.layers, args.dense_front, args.dense_back)]
-    dense = [(1, 0)] * args.layers
-
-    def one_pass(sched):
-        for P, mode in sched:
-            fps.skiparse2d_attn_fwd(q, k, v, P, mode, out=out)
-
-    def timed(sched, steps):
-        one_pass(sched)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            one_pass(sched)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        return max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
-
     for _ in range(args.warmup):
-        one_pass(hybrid)
-    h_ms = timed(hybrid, args.steps)
-    d_ms = timed(dense, max(1, args.steps // 2))
-    if fps.get_device_status() != 0:
-        raise SystemExit("device status error in the stack timing")
-    fl_h = sum(flops_padded(synth.custom(w.B, w.T, w.H, w.W, w.heads, w.d, P)) for P, _ in hybrid)
+        stack_pass(fps, q, k, v, [(w.P if p is None else p, m) for p, m in
+                                   stack_schedule(args.layers, args.dense_front, args.dense_back)],
+                   (torch.empty_like(q), torch.empty_like(q)))
+    st = time_stack(fps, w, q, k, v, args.layers, args.dense_front, args.dense_back, args.steps, world, dev,
+                    stream)
     if rank == 0:
         print(json.dumps({
-            "metric": "hybrid attention stack: ms per pass vs an all-dense stack (attention layers only)",
-            "value": round(h_ms, 2), "unit": "ms", "higher_is_better": False, "n_gpus": world,
+            "metric": "chained hybrid attention stack: ms per pass vs an all-dense stack (attention layers only)",
+            "value": st["ms_per_pass"], "unit": "ms", "higher_is_better": False, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "scaling": "weak", "dtype": "bf16",
-            "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16, the same inputs for every layer",
-            "config": {"workload": describe(w), "layers": args.layers,
-                       "dense_front": args.dense_front, "dense_back": args.dense_back,
-                       "sparse_layers": args.layers - args.dense_front - args.dense_back,
-                       "sparse_modes": "alternating token-wise / group-wise"},
-            "dense_stack_ms": round(d_ms, 2), "attention_speedup": round(d_ms / h_ms, 3),
-            "hybrid_tflops": round(fl_h / (h_ms / 1e3) / 1e12, 1), "gpu_launches_per_pass": args.layers,
+            "data": "synthetic: seeded N(0,1) q/k/v rounded to bf16",
+            "config": {"workload": describe(w), **{k_: st[k_] for k_ in ("layers", "dense_front", "dense_back",
+                                                                        "sparse_layers", "sparse_modes", "chaining")}},
+            "dense_stack_ms": st["dense_stack_ms"], "attention_speedup": st["attention_speedup"],
+            "hybrid_tflops": st["hybrid_tflops"], "gpu_launches_per_pass": args.layers,
         }), flush=True)
     if world > 1:
         torch.distributed.barrier()
@@ -753,7 +872,11 @@ def main(argv=None):
     ap.add_argument("--backward-steps", type=int, default=4)
     ap.add_argument("--rearrange-steps", type=int, default=10)
     ap.add_argument("--stack", action="store_true",
-                    help="time a hybrid stack of dense and alternating Skiparse-2D layers instead")
+                    help="time only the chained hybrid stack of dense and alternating Skiparse-2D layers")
+    ap.add_argument("--no-stack", action="store_true", help="skip the chained hybrid stack in the default run")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config table (480p, 768p P=2/3, 768p dense, 768p backward)")
+    ap.add_argument("--table-steps", type=int, default=4)
     ap.add_argument("--layers", type=int, default=40)
     ap.add_argument("--dense-front", type=int, default=4)
     ap.add_argument("--dense-back", type=int, default=4)
