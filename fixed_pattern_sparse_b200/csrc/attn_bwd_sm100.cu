@@ -9,13 +9,17 @@
 //   1. delta kernel: D = rowsum(dO o O) for every (token, head) row (HBM-bound);
 //   2. key-major kernel (KV = true): a CTA keeps one 128-key tile (K, V) and streams the class's
 //      query tiles (Q, dO, L, D): S^T = K Q^T and dP^T = V dO^T into TMEM; softmax warps make
-//      P^T and dS^T (bf16, over their own TMEM columns); dV += P^T dO and dK += dS^T Q accumulate
-//      in TMEM (TMEM: S^T, dP^T, dV, dK = 512 columns);
+//      P^T and dS^T (bf16, over the TMEM columns of S^T and dP^T); dV += P^T dO and
+//      dK += dS^T Q accumulate in TMEM (TMEM: S^T, dP^T, dV, dK = 512 columns);
 //   3. query-major kernel (KV = false): a CTA keeps one 128-query tile (Q, dO, L, D) and streams
-//      the class's key tiles (K, V): S, dP into TMEM, dS, then dQ += dS K in TMEM.
-// The MMA issuer runs one streamed tile ahead: the next tile's S (and dP) are computed while
-// the softmax warps work on the current tile.
+//      the class's key tiles (K, V): S, dP into TMEM, dS over dP's columns, then dQ += dS K.
 // No atomics: every gradient row is produced by exactly one CTA, so results are deterministic.
+//
+// Schedule. The MMA issuer runs one streamed tile ahead, so that the softmax of one tile overlaps
+// the tensor core's work on its neighbours. In the query-major kernel the softmax releases S's
+// columns as soon as it has read them, so S(j+1) is computed while it works on tile j; that kernel
+// keeps three key tiles in flight, because key tile j+1 is needed as soon as S(j) has been read
+// while tile j-1's slot is released only by its last reader, dQ(j-1).
 // Warp roles (13 warps): two softmax warpgroups (each owns 64 of the 128 streamed columns of
 // every TMEM row), four producer warps (16-byte cp.async gathers of class rows into the UMMA
 // swizzled layout, one pair per streamed tensor, 4-byte cp.async for L and D), one MMA warp
@@ -38,6 +42,7 @@ constexpr int kBwdProducers = 128;
 constexpr int kBwdMma = 12;
 constexpr int kBwdSoftmax = 256;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxSmem = 232448;  // 227 KB, the most a CTA may have
 
 template <int D, bool KV>
 struct BwdCfg : TileGeom<D> {
@@ -47,21 +52,30 @@ struct BwdCfg : TileGeom<D> {
     using G::TILE_BYTES;
     using G::LAYOUT;
     using G::KSTEPS;
-    // shared memory: two stationary tiles, two streamed slots of two tiles, L/D vectors
+    // ring slots of the two streamed tensors: B1 = Q (key-major) or K (query-major), B2 = dO or V
+    static constexpr int NS1 = KV ? 2 : 3, NS2 = 2;
+    // shared memory: two stationary tiles, the two rings, L/D vectors
     static constexpr int OFF_A1 = 0;
     static constexpr int OFF_A2 = TILE_BYTES;
-    static constexpr int OFF_B = 2 * TILE_BYTES;              // slot s: B1 at +2sT, B2 at +(2s+1)T
-    static constexpr int OFF_VEC = OFF_B + 4 * TILE_BYTES;    // [slot or stationary][L,D][128] fp32
-    static constexpr int VEC_BYTES = 2 * 2 * kTileRows * 4;
+    static constexpr int OFF_B1 = 2 * TILE_BYTES;
+    static constexpr int OFF_B2 = OFF_B1 + NS1 * TILE_BYTES;
+    static constexpr int OFF_VEC = OFF_B2 + NS2 * TILE_BYTES;  // [B1 slot or stationary][L,D][128] fp32
+    static constexpr int VEC_BYTES = (KV ? NS1 : 1) * 2 * kTileRows * 4;
     static constexpr int OFF_BAR = OFF_VEC + VEC_BYTES;
-    // B_FULL / B_EMPTY: [tensor (0: B1, 1: B2)][slot], index B_FULL + 2 * tensor + slot
-    static constexpr int B_STAT = 0, B_FULL = 1, B_EMPTY = 5, B_X1 = 9, B_X2 = 10, B_P = 11, B_DS = 12,
-                         B_ACC = 13, B_DRAIN = 14, B_X1FREE = 15, NBARS = 16;
+    static constexpr int B_STAT = 0, B_FULL1 = 1, B_EMPTY1 = B_FULL1 + NS1, B_FULL2 = B_EMPTY1 + NS1,
+                         B_EMPTY2 = B_FULL2 + NS2, B_X1 = B_EMPTY2 + NS2, B_X2 = B_X1 + 1, B_X1FREE = B_X2 + 1,
+                         B_P = B_X1FREE + 1, B_DS = B_P + 1, B_ACC = B_DS + 1,
+                         B_DRAIN = B_ACC + 1, NBARS = B_DRAIN + 1;
     static constexpr int OFF_TMEM_SLOT = OFF_BAR + 8 * NBARS;
     static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
     static constexpr int SMEM_USED = OFF_ABORT + 4;
-    static constexpr int SMEM_BYTES = SMEM_USED + 1024 > 118784 ? SMEM_USED + 1024 : 118784;
-    static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+    // + slack for 1024-byte alignment where it fits (the kernel checks the slack it got); at
+    // least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM even for small d
+    static constexpr int SMEM_BYTES =
+        SMEM_USED + 1024 > kMaxSmem ? kMaxSmem : (SMEM_USED + 1024 > 118784 ? SMEM_USED + 1024 : 118784);
+    // P^T (key-major) and dS (both kernels) are written in bf16 over the first half of each
+    // warpgroup's 64 score columns
+    static_assert(SMEM_USED + 256 <= kMaxSmem, "shared memory overflow");
     static constexpr uint32_t COL_X1 = 0, COL_X2 = 128, COL_ACC1 = 256, COL_ACC2 = 256 + D, NCOLS = 512;
     static_assert(COL_ACC2 + D <= NCOLS, "TMEM overflow");
 };
@@ -103,6 +117,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = ptx::smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw_base & 1023u)) & 1023u;
+    if (pad + C::SMEM_USED > static_cast<uint32_t>(C::SMEM_BYTES)) {
+        // the dynamic shared memory is not aligned well enough for this layout (uniform over the
+        // CTA, before any shared state): report it instead of running out of bounds
+        if (threadIdx.x == 0) atomicExch(p.status, kErrLaunch);
+        return;
+    }
     uint8_t* smem = smem_raw + pad;
     const uint32_t sbase = raw_base + pad;
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
@@ -116,15 +136,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(C::B_STAT), kBwdProducers);
-        for (int i = 0; i < 4; ++i) {
-            ptx::mbar_init(bar(C::B_FULL + i), kBwdProducers / 2);  // one producer pair per tensor
-            ptx::mbar_init(bar(C::B_EMPTY + i), 1);
+        for (int s = 0; s < C::NS1; ++s) {
+            ptx::mbar_init(bar(C::B_FULL1 + s), kBwdProducers / 2);  // one producer pair per tensor
+            ptx::mbar_init(bar(C::B_EMPTY1 + s), 1);
+        }
+        for (int s = 0; s < C::NS2; ++s) {
+            ptx::mbar_init(bar(C::B_FULL2 + s), kBwdProducers / 2);
+            ptx::mbar_init(bar(C::B_EMPTY2 + s), 1);
         }
         ptx::mbar_init(bar(C::B_X1), 1);
         ptx::mbar_init(bar(C::B_X2), 1);
+        ptx::mbar_init(bar(C::B_X1FREE), kBwdSoftmax);
         ptx::mbar_init(bar(C::B_P), kBwdSoftmax);
         ptx::mbar_init(bar(C::B_DS), kBwdSoftmax);
-        ptx::mbar_init(bar(C::B_X1FREE), kBwdSoftmax);
         ptx::mbar_init(bar(C::B_ACC), 1);
         ptx::mbar_init(bar(C::B_DRAIN), 1);
         *abort = 0;
@@ -147,10 +171,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
 
     if (warp >= kBwdProd0 && warp < kBwdProd0 + 4) {
         // ------------------------------------------------------------------ producers
-        // Pair 0 (warps 8-9) copies the first tensor of every tile (and the L/D statistics),
-        // pair 1 (warps 10-11) the second; within a pair, warp pw copies rows [64pw, 64pw+64).
+        // Pair 0 (warps 8-9) copies the first streamed tensor (and the L/D statistics), pair 1
+        // (warps 10-11) the second; within a pair, warp pw copies rows [64pw, 64pw+64).
         const int pair = (warp - kBwdProd0) >> 1;
         const int pw = (warp - kBwdProd0) & 1;
+        const int ns = pair ? C::NS2 : C::NS1;
         const TileRows ta = tile_rows(rows, first, n_c, pw, lane, p.nrows, p.status);
         load_tile_rows<D>(sbase + (pair ? C::OFF_A2 : C::OFF_A1), pair ? g_a2 : g_a1, ta, pw, lane);
         if (!KV && pair == 0) {  // the stationary queries' L and D
@@ -160,19 +185,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         cp_async_arrive_noinc(bar(C::B_STAT));
         bool ok = true;
         for (int j = 0; j < nstream; ++j) {
-            const int s = j & 1;
-            if (j >= 2) {
+            const int s = j % ns;
+            if (j >= ns) {
                 int w_ok = 1;
-                if (lane == 0) w_ok = ptx::mbar_wait(bar(C::B_EMPTY + 2 * pair + s), ((j >> 1) - 1) & 1, abort, lim);
+                if (lane == 0)
+                    w_ok = ptx::mbar_wait(bar((pair ? C::B_EMPTY2 : C::B_EMPTY1) + s), ((j / ns) - 1) & 1, abort, lim);
                 w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
                 if (!w_ok) {
                     ok = false;
                     break;
                 }
             }
-            const uint32_t slot = sbase + C::OFF_B + 2 * s * C::TILE_BYTES;
             const TileRows tr = tile_rows(rows, j * kTileRows, n_c, pw, lane, p.nrows, p.status);
-            load_tile_rows<D>(slot + (pair ? C::TILE_BYTES : 0), pair ? g_b2 : g_b1, tr, pw, lane);
+            load_tile_rows<D>(sbase + (pair ? C::OFF_B2 : C::OFF_B1) + s * C::TILE_BYTES, pair ? g_b2 : g_b1, tr,
+                              pw, lane);
             if (KV && pair == 0) {  // the streamed queries' L and D
                 const uint32_t v = sbase + C::OFF_VEC + s * 2 * 4 * kTileRows;
                 load_vec(v, p.lse, tr, pw, lane);
@@ -181,7 +207,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             // completes when this tile has landed; test hook: one thread of the key-major kernel
             // never signals the first streamed tile
             if (!(KV && p.fault == 1 && j == 0 && pair == 0 && pw == 0 && lane == 0))
-                cp_async_arrive_noinc(bar(C::B_FULL + 2 * pair + s));
+                cp_async_arrive_noinc(bar((pair ? C::B_FULL2 : C::B_FULL1) + s));
         }
         cp_async_commit();
         cp_async_wait<0>();  // no copy of this thread outlives it
@@ -193,80 +219,79 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             const uint32_t idesc_acc = ptx::idesc_bf16_f32(kTileRows, D, true);
             const uint64_t a1 = ptx::smem_desc(sbase + C::OFF_A1, 16, 8 * C::SW, C::LAYOUT);
             const uint64_t a2 = ptx::smem_desc(sbase + C::OFF_A2, 16, 8 * C::SW, C::LAYOUT);
-            const uint64_t bk0 = ptx::smem_desc(sbase + C::OFF_B, 16, 8 * C::SW, C::LAYOUT);
-            const uint64_t bm0 = ptx::smem_desc(sbase + C::OFF_B, C::BOX_BYTES, 8 * C::SW, C::LAYOUT);
-            auto x_mma = [&](uint64_t a, uint64_t bk, uint32_t d_tmem) {   // D = A B^T over d
+            // streamed tiles read K-major (as the B of S, dP) or MN-major (as the B of dV, dK, dQ)
+            auto bk = [&](int off) { return ptx::smem_desc(sbase + off, 16, 8 * C::SW, C::LAYOUT); };
+            auto bm = [&](int off) { return ptx::smem_desc(sbase + off, C::BOX_BYTES, 8 * C::SW, C::LAYOUT); };
+            auto x_mma = [&](uint64_t a, uint64_t b, uint32_t d_tmem) {   // D = A B^T over d
 #pragma unroll
                 for (int kk = 0; kk < C::KSTEPS; ++kk) {
                     const uint32_t off = C::kstep_off(kk) >> 4;
-                    ptx::mma_ss(d_tmem, a + off, bk + off, idesc_x, kk > 0 ? 1u : 0u);
+                    ptx::mma_ss(d_tmem, a + off, b + off, idesc_x, kk > 0 ? 1u : 0u);
                 }
             };
-            auto acc_mma = [&](uint32_t a_col, uint64_t bm, uint32_t d_tmem, bool acc) {  // D += A B
+            // D += A B over the 128 streamed rows, A from TMEM (P^T, dS^T or dS, half-packed columns)
+            auto acc_mma = [&](uint32_t a_col, uint64_t b, uint32_t d_tmem, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < kTileRows / 16; ++kk)
-                    ptx::mma_ts(d_tmem, tmem + a_col + half_packed_col(kk), bm + ((kk * 16 * C::SW) >> 4),
+                    ptx::mma_ts(d_tmem, tmem + a_col + half_packed_col(kk), b + ((kk * 16 * C::SW) >> 4),
                                 idesc_acc, (acc || kk > 0) ? 1u : 0u);
             };
-            // Issue order per streamed tile j, so that the softmax of one tile overlaps the tensor
-            // core's work on its neighbours (every MMA below reuses a TMEM region only after the
-            // MMA that last read it, in issue order):
-            //   key-major  : dV(j) [P(j)], X1(j+1), dK(j) [dS(j)], X2(j+1)
-            //   query-major: X1(j+1) [S(j) read by the softmax], dQ(j) [dS(j)], X2(j+1)
-            auto issue_x1 = [&](int j) -> bool {   // S (or S^T) of streamed tile j
-                const int s = j & 1;
-                if (!ptx::mbar_wait(bar(C::B_FULL + s), (j >> 1) & 1, abort, lim)) return false;  // B1
+            auto b1_off = [&](int j) { return C::OFF_B1 + (j % C::NS1) * C::TILE_BYTES; };
+            auto b2_off = [&](int j) { return C::OFF_B2 + (j % C::NS2) * C::TILE_BYTES; };
+            // S (or S^T) of streamed tile j into X1; dP (or dP^T) into X2
+            auto issue_x1 = [&](int j) {
                 fence_proxy_async();  // the cp.async data, observed through the barrier, for the MMA
                 ptx::tc_fence_after();
-                x_mma(a1, bk0 + ((2 * s * C::TILE_BYTES) >> 4), tmem + C::COL_X1);
+                x_mma(a1, bk(b1_off(j)), tmem + C::COL_X1);
                 ptx::mma_commit(bar(C::B_X1));
-                return true;
             };
-            auto issue_x2 = [&](int j) -> bool {   // dP (or dP^T) of streamed tile j
-                const int s = j & 1;
-                if (!ptx::mbar_wait(bar(C::B_FULL + 2 + s), (j >> 1) & 1, abort, lim)) return false;  // B2
+            auto issue_x2 = [&](int j) {
                 fence_proxy_async();
                 ptx::tc_fence_after();
-                x_mma(a2, bk0 + (((2 * s + 1) * C::TILE_BYTES) >> 4), tmem + C::COL_X2);
+                x_mma(a2, bk(b2_off(j)), tmem + C::COL_X2);
                 ptx::mma_commit(bar(C::B_X2));
-                if (!KV) ptx::mma_commit(bar(C::B_EMPTY + 2 + s));  // V_j: dP was its last reader
-                return true;
+                if (!KV) ptx::mma_commit(bar(C::B_EMPTY2 + j % C::NS2));  // V_j: dP was its last reader
             };
             bool ok = ptx::mbar_wait(bar(C::B_STAT), 0, abort, lim);
-            fence_proxy_async();
-            ok = ok && issue_x1(0) && issue_x2(0);
+            if (ok) fence_proxy_async();
+            ok = ok && ptx::mbar_wait(bar(C::B_FULL1), 0, abort, lim);
+            if (ok) issue_x1(0);
+            ok = ok && ptx::mbar_wait(bar(C::B_FULL2), 0, abort, lim);
+            if (ok) issue_x2(0);
+            auto wait = [&](int b, int parity) { return ptx::mbar_wait(bar(b), parity, abort, lim); };
+            // Per streamed tile j, in a fixed order (each wait suspends the thread in hardware until
+            // its phase completes):
+            //   key-major  : dV(j) once P^T(j) is in TMEM, S^T(j+1) (over the columns dV(j) has just
+            //                read), dK(j) once dS^T(j) is in TMEM, dP^T(j+1) (over dS^T(j)'s columns)
+            //   query-major: S(j+1) once the softmax has read S(j), dQ(j) once dS(j) is in TMEM,
+            //                dP(j+1) (over dS(j)'s columns)
             for (int j = 0; ok && j < nstream; ++j) {
-                const int s = j & 1;
                 const bool more = j + 1 < nstream;
-                const uint64_t b1m = bm0 + ((2 * s * C::TILE_BYTES) >> 4);
-                const uint64_t b2m = bm0 + (((2 * s + 1) * C::TILE_BYTES) >> 4);
                 if (KV) {
-                    if (!ptx::mbar_wait(bar(C::B_P), j & 1, abort, lim)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = wait(C::B_P, j & 1);
+                    if (!ok) break;
                     ptx::tc_fence_after();
-                    acc_mma(C::COL_X1, b2m, tmem + C::COL_ACC1, j > 0);   // dV += P^T dO
-                    ptx::mma_commit(bar(C::B_EMPTY + 2 + s));             // dO_j: dV was its last reader
-                } else if (!ptx::mbar_wait(bar(C::B_X1FREE), j & 1, abort, lim)) {
-                    ok = false;
-                    break;
+                    acc_mma(C::COL_X1, bm(b2_off(j)), tmem + C::COL_ACC1, j > 0);  // dV += P^T dO
+                    ptx::mma_commit(bar(C::B_EMPTY2 + j % C::NS2));                 // dO_j: dV was its last reader
+                } else {
+                    ok = wait(C::B_X1FREE, j & 1);
+                    if (!ok) break;
                 }
-                if (more && !issue_x1(j + 1)) {
-                    ok = false;
-                    break;
+                if (more) {
+                    ok = wait(C::B_FULL1 + (j + 1) % C::NS1, ((j + 1) / C::NS1) & 1);
+                    if (!ok) break;
+                    issue_x1(j + 1);
                 }
-                if (!ptx::mbar_wait(bar(C::B_DS), j & 1, abort, lim)) {
-                    ok = false;
-                    break;
-                }
+                ok = wait(C::B_DS, j & 1);
+                if (!ok) break;
                 ptx::tc_fence_after();
                 // key-major: dK += dS^T Q ; query-major: dQ += dS K
-                acc_mma(C::COL_X2, b1m, tmem + (KV ? C::COL_ACC2 : C::COL_ACC1), j > 0);
-                ptx::mma_commit(bar(C::B_EMPTY + s));  // B1 of tile j: dK / dQ was its last reader
-                if (more && !issue_x2(j + 1)) {
-                    ok = false;
-                    break;
+                acc_mma(C::COL_X2, bm(b1_off(j)), tmem + (KV ? C::COL_ACC2 : C::COL_ACC1), j > 0);
+                ptx::mma_commit(bar(C::B_EMPTY1 + j % C::NS1));  // B1 of tile j: its last reader
+                if (more) {
+                    ok = wait(C::B_FULL2 + (j + 1) % C::NS2, ((j + 1) / C::NS2) & 1);
+                    if (!ok) break;
+                    issue_x2(j + 1);
                 }
             }
             if (ok) {
@@ -274,6 +299,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             } else {
                 record_abort(abort, p.status);
             }
+            // every MMA issued by this thread must finish before TMEM is released
             ptx::mma_commit(bar(C::B_DRAIN));
             volatile int never = 0;
             ptx::mbar_wait(bar(C::B_DRAIN), 0, &never, lim);
@@ -290,7 +316,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
         float row_l2 = 0.f, row_d = 0.f;
         bool ok = true;
         for (int j = 0; j < nstream; ++j) {
-            const int s = j & 1;
+            const int s1 = j % C::NS1;
             const int valid = n_c - j * kTileRows;     // streamed rows in this tile (>= 1)
             // every wait of a softmax warp is made uniform over the warp: the tcgen05.ld/st below
             // are .sync.aligned and need all 32 lanes
@@ -300,8 +326,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
             }
             ptx::tc_fence_after();
             // the L/D vectors were written by the producers' cp.async: observe their barrier too
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(KV ? bar(C::B_FULL + s) : bar(C::B_STAT),
-                                                        KV ? (j >> 1) & 1 : 0, abort, lim))) {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(KV ? bar(C::B_FULL1 + s1) : bar(C::B_STAT),
+                                                        KV ? (j / C::NS1) & 1 : 0, abort, lim))) {
                 ok = false;
                 break;
             }
@@ -309,7 +335,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
                 row_l2 = vecs[row] * kLog2e;
                 row_d = vecs[kTileRows + row];
             }
-            const float* col_l = vecs + s * 2 * kTileRows + 64 * h;   // key-major: per column
+            const float* col_l = vecs + s1 * 2 * kTileRows + 64 * h;   // key-major: per column
             const float* col_d = col_l + kTileRows;
             float pr[64];
             {

@@ -114,7 +114,7 @@ struct RearrangeParams {
 };
 
 // Status codes (mirror include/skiparse.h).
-enum : int { kOk = 0, kErrTimeout = 5, kErrBounds = 6 };
+enum : int { kOk = 0, kErrLaunch = 4, kErrTimeout = 5, kErrBounds = 6 };
 
 // The row index a global load may use: `row` itself, or (debug builds, row outside
 // [0, nrows)) row 0 after recording kErrBounds.
