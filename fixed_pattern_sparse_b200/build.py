@@ -21,7 +21,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libskiparse.so")
 DEBUG_LIB = os.path.join(HERE, "libskiparse_debug.so")
 SOURCES = ["skiparse_api.cu", "attn_fwd_sm100.cu", "attn_bwd_sm100.cu", "rearrange.cu", "no_alloc.cu",
-           "host_pipeline.cu"]
+           "host_pipeline.cu", "diag_sm100.cu"]
 HEADERS = ["ptx_sm100.cuh", "skiparse_internal.cuh", "attn_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

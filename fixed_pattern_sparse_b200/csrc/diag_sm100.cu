@@ -1,0 +1,116 @@
+// diag_sm100.cu -- diagnostic microbenchmark of the tensor-core issue patterns the attention
+// kernels use (no counterpart on the pages): how many SM clocks a tcgen05.mma of each shape takes
+// when one thread issues a long unrolled stream of them, the way the kernels' MMA warp does.
+//
+// Every CTA (one per SM: it allocates all 512 TMEM columns and holds 100 KB of shared memory)
+// fills an A tile (128 x 128 bf16) and a B tile (256 x 128 bf16) in shared memory, then lane 0 of
+// warp 0 issues `groups` groups of 8 K-steps (K = 16 each) into one fp32 accumulator in TMEM,
+// commits, and waits (bounded) for completion; the SM clocks from the first issue to completion
+// go to clocks[blockIdx.x]. Patterns:
+//   0: A and B from shared memory, M = 128, N = 128  (S = Q K^T)
+//   1: A from TMEM,                M = 128, N = 128  (O += P V with P in TMEM)
+//   2: A and B from shared memory, M = 128, N = 256
+//   3: A and B from shared memory, M = 128, N = 64
+// Work per group: 8 x 2 x 128 x N x 16 FLOP. A wait that runs out leaves clocks = -1.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "attn_common.cuh"
+
+namespace skiparse {
+namespace {
+
+constexpr int kDiagBox = 128 * 128;           // 128 rows x 64 bf16, 128-byte swizzle
+constexpr int kDiagA = 2 * kDiagBox;          // 128 x 128 bf16
+constexpr int kDiagB = 2 * 256 * 128;         // 256 x 128 bf16
+constexpr int kDiagSmem = 100 * 1024;         // > 227 KB / 3: at most two CTAs per SM by shared
+                                              // memory; TMEM (512 columns each) admits one
+
+template <int PATTERN>
+__global__ void __launch_bounds__(128, 1) skiparse_mma_rate_kernel(long long* clocks, int groups,
+                                                                    unsigned long long wait_ns) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) unsigned long long done_bar;
+    __shared__ uint32_t tmem_slot;
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t a_s = raw + pad, b_s = a_s + kDiagA;
+    // bf16 1.0 / 0.5 / -1.0 / 0.25 patterns: finite values, the contents do not matter
+    for (int i = threadIdx.x; i < (kDiagA + kDiagB) / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0x3f803f80u, 0x3f003f00u, 0xbf80bf80u, 0x3e803e80u);
+    const uint32_t bar = ptx::smem_u32(&done_bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    if (threadIdx.x < 32) {
+        ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), 512);
+        ptx::tmem_relinquish();
+    }
+    fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    if (threadIdx.x == 0) {
+        const uint64_t ad = ptx::smem_desc(a_s, 16, 1024, 2);
+        const uint64_t bd = ptx::smem_desc(b_s, 16, 1024, 2);
+        constexpr int N = PATTERN == 2 ? 256 : PATTERN == 3 ? 64 : 128;
+        constexpr int B_BOX = 256 * 128;  // B boxes are laid out for 256 rows
+        const uint32_t idesc = ptx::idesc_bf16_f32(128, N, false);
+        const long long t0 = clock64();
+        for (int g = 0; g < groups; ++g) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t a_off = ((kk / 4) * kDiagBox + (kk % 4) * 32) >> 4;
+                const uint32_t b_off = ((kk / 4) * B_BOX + (kk % 4) * 32) >> 4;
+                if (PATTERN == 1) {
+                    // A: 128 x 16 bf16 in TMEM columns 384 + 8 kk (never written: the values do
+                    // not matter for timing), accumulator at column 0
+                    ptx::mma_ts(tmem, tmem + 384 + 8 * kk, bd + b_off, idesc, (g | kk) != 0);
+                } else {
+                    ptx::mma_ss(tmem, ad + a_off, bd + b_off, idesc, (g | kk) != 0);
+                }
+            }
+        }
+        ptx::mma_commit(bar);
+        volatile int never = 0;
+        const bool ok = ptx::mbar_wait(bar, 0, &never, wait_ns);
+        clocks[blockIdx.x] = ok ? clock64() - t0 : -1;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int PATTERN>
+int launch_pattern(long long* clocks, int ctas, int groups, unsigned long long wait_ns, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(skiparse_mma_rate_kernel<PATTERN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kDiagSmem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    skiparse_mma_rate_kernel<PATTERN><<<ctas, 128, kDiagSmem, st>>>(clocks, groups, wait_ns);
+    return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+static_assert(kDiagA + kDiagB + 1024 <= kDiagSmem, "diagnostic shared memory");
+
+int launch_mma_rate(long long* clocks, int ctas, int pattern, int groups, unsigned long long wait_ns,
+                    void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (pattern) {
+        case 0: return launch_pattern<0>(clocks, ctas, groups, wait_ns, st);
+        case 1: return launch_pattern<1>(clocks, ctas, groups, wait_ns, st);
+        case 2: return launch_pattern<2>(clocks, ctas, groups, wait_ns, st);
+        case 3: return launch_pattern<3>(clocks, ctas, groups, wait_ns, st);
+        default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+}
+
+}  // namespace skiparse

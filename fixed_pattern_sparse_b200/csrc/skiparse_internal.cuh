@@ -146,5 +146,7 @@ int launch_attn_bwd(const BwdParams& p, const Geometry& g, void* stream);
 int launch_rearrange(const RearrangeParams& p, int kind, void* stream);  // 0 fwd, 1 inverse, 2 switch
 int attn_smem_bytes(int d);
 int launch_exp2(const float* x, float* y, long long n, void* stream);
+int launch_mma_rate(long long* clocks, int ctas, int pattern, int groups, unsigned long long wait_ns,
+                    void* stream);
 
 }  // namespace skiparse

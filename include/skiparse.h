@@ -318,6 +318,23 @@ SKIPARSE_API int skiparse_debug_shrink_bounds(long long rows);
 SKIPARSE_API int skiparse_debug_exp2(const float* x, float* y, long long n, int method,
                                      skiparse_stream_t stream);
 
+/*
+ * Diagnostic (no counterpart on the pages): the tensor-core rate behind the kernels' design.
+ * Launches n_clocks CTAs (pass the SM count: one per SM); in each, one thread issues `groups`
+ * groups of 8 tcgen05.mma K-steps (K = 16, bf16 in, fp32 accumulator in TMEM) in an unrolled
+ * stream, as the attention kernels' MMA warp does, and writes the SM clocks from the first issue
+ * to completion to clocks[cta] (-1 if its bounded wait ran out). Patterns: 0 = A and B in shared
+ * memory, M = 128, N = 128; 1 = A in TMEM, M = N = 128; 2 = shared memory, N = 256;
+ * 3 = shared memory, N = 64. One group is 8 x 2 x 128 x N x 16 FLOP; the nominal dense bf16 rate
+ * of an SM is 8192 FLOP per clock.
+ *   clocks : device pointer to n_clocks int64, 8-byte aligned. 1 <= n_clocks <= 4096,
+ *            1 <= groups <= 65536, 0 <= pattern <= 3.
+ * Asynchronous on `stream`. Returns SKIPARSE_OK, SKIPARSE_ERR_INVALID_ARG, _UNSUPPORTED,
+ * _MISALIGNED or SKIPARSE_ERR_CUDA.
+ */
+SKIPARSE_API int skiparse_debug_mma_rate(int pattern, int groups, long long* clocks, int n_clocks,
+                                         skiparse_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

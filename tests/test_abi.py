@@ -149,6 +149,14 @@ def test_noalloc_backward_rejects_bad_arguments_before_any_cuda_call(L):
     assert f(*([FAKE] * 9), 1, 1, 1, (1 << 22) + 1, 1, 32, 2, 0, None) == 2  # beyond the workspace
 
 
+def test_mma_rate_diagnostic_rejects_bad_arguments_synchronously(L):
+    assert L.skiparse_debug_mma_rate(4, 8, FAKE, 148, None) == 1
+    assert L.skiparse_debug_mma_rate(0, 0, FAKE, 148, None) == 1
+    assert L.skiparse_debug_mma_rate(0, 8, 0, 148, None) == 1
+    assert L.skiparse_debug_mma_rate(0, 1 << 20, FAKE, 148, None) == 2
+    assert L.skiparse_debug_mma_rate(0, 8, FAKE + 4, 148, None) == 3
+
+
 def test_rearrange_rejects_bad_arguments_synchronously(L):
     assert L.skiparse_rearrange(0, FAKE, 1, 2, 8, 8, 2, 32, 2, 0, None) == 1
     assert L.skiparse_rearrange(FAKE, FAKE + 4, 1, 2, 8, 8, 2, 32, 2, 0, None) == 3
