@@ -73,9 +73,9 @@ struct BwdCfg : TileGeom<D> {
     // least 116 KB so that one CTA (and its 512 TMEM columns) owns an SM even for small d
     static constexpr int SMEM_BYTES =
         SMEM_USED + 1024 > kMaxSmem ? kMaxSmem : (SMEM_USED + 1024 > 118784 ? SMEM_USED + 1024 : 118784);
-    // P^T (key-major) and dS (both kernels) are written in bf16 over the first half of each
-    // warpgroup's 64 score columns
     static_assert(SMEM_USED + 256 <= kMaxSmem, "shared memory overflow");
+    // TMEM: X1 = S (or S^T), X2 = dP (or dP^T); P^T (key-major) and dS (both kernels) are written
+    // in bf16 over the first half of each warpgroup's 64 columns of X1 and X2
     static constexpr uint32_t COL_X1 = 0, COL_X2 = 128, COL_ACC1 = 256, COL_ACC2 = 256 + D, NCOLS = 512;
     static_assert(COL_ACC2 + D <= NCOLS, "TMEM overflow");
 };
