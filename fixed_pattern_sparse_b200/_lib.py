@@ -38,6 +38,7 @@ SIGNATURES = {
     "skiparse_debug_shrink_bounds": (_I, [_LL]),
     "skiparse_debug_exp2": (_I, [_VP, _VP, _LL, _I, _VP]),
     "skiparse_debug_mma_rate": (_I, [_I, _I, _VP, _I, _VP]),
+    "skiparse_debug_softmax_rate": (_I, [_I, _I, _VP, _I, _VP]),
     "skiparse1d_attn_fwd": (_I, [_VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse1d_attn_fwd_lse": (_I, [_VP, _VP, _VP, _VP, _VP] + [_I] * 8 + [_VP]),
     "skiparse1d_attn_bwd": (_I, [_VP] * 10 + [_I] * 8 + [_VP]),

@@ -12,6 +12,12 @@
 //   2: A and B from shared memory, M = 128, N = 256
 //   3: A and B from shared memory, M = 128, N = 64
 // Work per group: 8 x 2 x 128 x N x 16 FLOP. A wait that runs out leaves clocks = -1.
+//
+// A second diagnostic times the forward softmax's exponential loop alone (no tensor core, no
+// loads): skiparse_softmax_rate_kernel runs, in every warp of a CTA that owns its SM, `reps`
+// passes over 64 scores per thread of the loop body the attention softmax uses (exponent by
+// FFMA, ex2.approx, four running sums, bf16 pack), with 1, 2 or 4 warps per SM sub-partition,
+// and writes each warp's SM clocks to clocks[cta * warps + warp].
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -97,9 +103,57 @@ int launch_pattern(long long* clocks, int ctas, int groups, unsigned long long w
     return static_cast<int>(cudaGetLastError());
 }
 
+__global__ void __launch_bounds__(512, 1) skiparse_softmax_rate_kernel(long long* clocks, int reps, float sl2) {
+    // scores of a plausible range (the values do not change the instruction stream)
+    float sc[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) sc[e] = -0.03125f * static_cast<float>((threadIdx.x * 7 + e * 3) & 63);
+    float neg = -1.f;
+    float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+    uint32_t packs = 0;
+    __syncthreads();
+    const long long t0 = clock64();
+    for (int r = 0; r < reps; ++r) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const float p0 = ptx::ex2_approx(fmaf(sc[2 * e], sl2, neg));
+            const float p1 = ptx::ex2_approx(fmaf(sc[2 * e + 1], sl2, neg));
+            if (e & 1) {
+                sum2 += p0;
+                sum3 += p1;
+            } else {
+                sum0 += p0;
+                sum1 += p1;
+            }
+            packs ^= ptx::pack_bf16x2(p0, p1);
+        }
+        neg -= 1.0e-7f;  // a new exponent offset per pass, as a new running maximum would be
+    }
+    // the results are complete before the second clock read (the compiler may not move the
+    // loop's work past it)
+    asm volatile("" ::"f"(sum0), "f"(sum1), "f"(sum2), "f"(sum3), "r"(packs) : "memory");
+    const long long t1 = clock64();
+    // the results feed the output (a NaN pattern no finite sum produces adds one clock), so the
+    // loop cannot be removed
+    const uint32_t bits = __float_as_uint((sum0 + sum1) + (sum2 + sum3)) ^ packs;
+    if ((threadIdx.x & 31) == 0)
+        clocks[static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)] =
+            t1 - t0 + (bits == 0x7fc00001u ? 1 : 0);
+}
+
 }  // namespace
 
 static_assert(kDiagA + kDiagB + 1024 <= kDiagSmem, "diagnostic shared memory");
+
+int launch_softmax_rate(long long* clocks, int ctas, int warps_per_subpartition, int reps, void* stream) {
+    cudaError_t e = cudaFuncSetAttribute(skiparse_softmax_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDiagSmem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    // kDiagSmem of (unused) dynamic shared memory: one CTA per SM
+    skiparse_softmax_rate_kernel<<<ctas, 128 * warps_per_subpartition, kDiagSmem, static_cast<cudaStream_t>(stream)>>>(
+        clocks, reps, 1.4426950408889634f * 0.08838834764831845f);
+    return static_cast<int>(cudaGetLastError());
+}
 
 int launch_mma_rate(long long* clocks, int ctas, int pattern, int groups, unsigned long long wait_ns,
                     void* stream) {

@@ -217,6 +217,16 @@ int skiparse_debug_mma_rate(int pattern, int groups, long long* clocks, int n_cl
     return e == 0 ? SKIPARSE_OK : cuda_fail(e);
 }
 
+int skiparse_debug_softmax_rate(int warps_per_subpartition, int reps, long long* clocks, int n_ctas,
+                                skiparse_stream_t stream) {
+    const int wps = warps_per_subpartition;
+    if ((wps != 1 && wps != 2 && wps != 4) || reps < 1 || n_ctas < 1 || !clocks) return SKIPARSE_ERR_INVALID_ARG;
+    if (reps > 65536 || n_ctas > 1024) return SKIPARSE_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(clocks) & 7u) return SKIPARSE_ERR_MISALIGNED;
+    const int e = skiparse::launch_softmax_rate(clocks, n_ctas, wps, reps, stream);
+    return e == 0 ? SKIPARSE_OK : cuda_fail(e);
+}
+
 int skiparse_get_device_status(skiparse_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {

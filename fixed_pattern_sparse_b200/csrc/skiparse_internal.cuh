@@ -148,5 +148,6 @@ int attn_smem_bytes(int d);
 int launch_exp2(const float* x, float* y, long long n, void* stream);
 int launch_mma_rate(long long* clocks, int ctas, int pattern, int groups, unsigned long long wait_ns,
                     void* stream);
+int launch_softmax_rate(long long* clocks, int ctas, int warps_per_subpartition, int reps, void* stream);
 
 }  // namespace skiparse

@@ -335,6 +335,21 @@ SKIPARSE_API int skiparse_debug_exp2(const float* x, float* y, long long n, int 
 SKIPARSE_API int skiparse_debug_mma_rate(int pattern, int groups, long long* clocks, int n_clocks,
                                          skiparse_stream_t stream);
 
+/*
+ * Diagnostic (no counterpart on the pages): the rate of the forward softmax's exponential loop,
+ * with no tensor core or loads beside it. Launches n_ctas CTAs (pass the SM count: one
+ * per SM) of 4 x warps_per_subpartition warps; every warp runs `reps` passes of the softmax's
+ * loop body over 64 scores per thread (exponent by FFMA, ex2.approx, four running sums, bf16
+ * pack: 64 exponentials per thread per pass) and writes its SM clocks to
+ * clocks[cta * 4 * warps_per_subpartition + warp].
+ *   clocks : device pointer to n_ctas * 4 * warps_per_subpartition int64, 8-byte aligned.
+ *            warps_per_subpartition in {1, 2, 4}, 1 <= reps <= 65536, 1 <= n_ctas <= 1024.
+ * Asynchronous on `stream`. Returns SKIPARSE_OK, SKIPARSE_ERR_INVALID_ARG, _UNSUPPORTED,
+ * _MISALIGNED or SKIPARSE_ERR_CUDA.
+ */
+SKIPARSE_API int skiparse_debug_softmax_rate(int warps_per_subpartition, int reps, long long* clocks,
+                                             int n_ctas, skiparse_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -257,3 +257,14 @@ int main(void) {
     # rows h with (h div 2) mod 2 = 1 below 45 (11 blocks of 4 rows x 2) and 40 of the 80 columns
     assert out[0] == "48" and out[1] == str(21 * 24 * 40) and out[2] == str(21 * 22 * 40)
     assert out[3] == "SKIPARSE_ERR_TIMEOUT" and out[4] == "SKIPARSE_ERR_BOUNDS"
+
+
+def test_softmax_rate_diagnostic_rejects_bad_arguments_synchronously(L):
+    assert L.skiparse_debug_softmax_rate(3, 8, FAKE, 148, None) == 1
+    assert L.skiparse_debug_softmax_rate(0, 8, FAKE, 148, None) == 1
+    assert L.skiparse_debug_softmax_rate(2, 0, FAKE, 148, None) == 1
+    assert L.skiparse_debug_softmax_rate(2, 8, 0, 148, None) == 1
+    assert L.skiparse_debug_softmax_rate(2, 8, FAKE, 0, None) == 1
+    assert L.skiparse_debug_softmax_rate(2, 1 << 20, FAKE, 148, None) == 2
+    assert L.skiparse_debug_softmax_rate(2, 8, FAKE, 2000, None) == 2
+    assert L.skiparse_debug_softmax_rate(2, 8, FAKE + 4, 148, None) == 3
