@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured on: a changed kernel reports null until it is captured again.
 KNOWN_TRAFFIC = {
     # 2.33 GB read + 0.756 GB written (q, k, v read once, out written once)
-    "c9c40496fc257c10": 3.086e9,
+    "e6281fdc8f37edc8": 3.086e9,
 }
 
 ATTN_SOURCES = ["fixed_pattern_sparse_b200/csrc/attn_fwd_sm100.cu",
