@@ -408,9 +408,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) skiparse_attn_bwd_kernel(const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = 8 * e4 + 2 * e;  // column inside this 32-column chunk
-                        const float s0 = pr[32 * g + c] * (__uint_as_float(dv[c]) - dcol[2 * e]);
-                        const float s1 = pr[32 * g + c + 1] * (__uint_as_float(dv[c + 1]) - dcol[2 * e + 1]);
-                        pk[4 * e4 + e] = ptx::pack_bf16x2(s0, s1);
+                        // two columns per instruction (packed f32x2): dP - D (exact, as an FMA with
+                        // -1), then P * (dP - D). This loop has no MUFU work to stall on, and while
+                        // it runs the MMA thread on the same sub-partition gets few issue slots, so
+                        // fewer instructions here shorten the tensor core's wait as well.
+                        const float2 x = __ffma2_rn(make_float2(dcol[2 * e], dcol[2 * e + 1]), make_float2(-1.f, -1.f),
+                                                    make_float2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])));
+                        const float2 sv = __fmul2_rn(make_float2(pr[32 * g + c], pr[32 * g + c + 1]), x);
+                        pk[4 * e4 + e] = ptx::pack_bf16x2(sv.x, sv.y);
                     }
                 }
                 ptx::tmem_st16(x2 + 16 * g, pk);
