@@ -11,6 +11,11 @@
 //   1: A from TMEM,                M = 128, N = 128  (O += P V with P in TMEM)
 //   2: A and B from shared memory, M = 128, N = 256
 //   3: A and B from shared memory, M = 128, N = 64
+//   4, 5, 6: pattern 0 while 8 more warps of the CTA (2 per SM sub-partition, including the
+//      issuing thread's) run, until the stream is done, a loop of independent FFMA chains (4),
+//      the backward's dS arithmetic (5: FADD, FMUL, bf16 pack, no MUFU) or the forward
+//      softmax's exponential loop (6: FFMA, ex2, FADD, bf16 pack): how much the tensor pipe
+//      loses when its issuing thread shares a sub-partition with warps that never stall.
 // Work per group: 8 x 2 x 128 x N x 16 FLOP. A wait that runs out leaves clocks = -1.
 //
 // A second diagnostic times the forward softmax's exponential loop alone (no tensor core, no
@@ -141,6 +146,110 @@ __global__ void __launch_bounds__(512, 1) skiparse_softmax_rate_kernel(long long
             t1 - t0 + (bits == 0x7fc00001u ? 1 : 0);
 }
 
+// Patterns 4-6: warp 0's lane 0 issues pattern 0's stream; warps 4-11 run background loop BG
+// (0 FFMA chains, 1 dS arithmetic, 2 exponential loop) until the stream has completed (a flag
+// in shared memory; at most 1 << 20 passes).
+template <int BG>
+__global__ void __launch_bounds__(384, 1) skiparse_mma_contended_kernel(long long* clocks, int groups,
+                                                                         unsigned long long wait_ns) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) unsigned long long done_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile int stop;
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t a_s = raw + pad, b_s = a_s + kDiagA;
+    for (int i = threadIdx.x; i < (kDiagA + kDiagB) / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0x3f803f80u, 0x3f003f00u, 0xbf80bf80u, 0x3e803e80u);
+    const uint32_t bar = ptx::smem_u32(&done_bar);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+        stop = 0;
+    }
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), 512);
+        ptx::tmem_relinquish();
+    }
+    fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    if (warp == 0) {
+        if (threadIdx.x == 0) {
+            const uint64_t ad = ptx::smem_desc(a_s, 16, 1024, 2);
+            const uint64_t bd = ptx::smem_desc(b_s, 16, 1024, 2);
+            constexpr int B_BOX = 256 * 128;
+            const uint32_t idesc = ptx::idesc_bf16_f32(128, 128, false);
+            const long long t0 = clock64();
+            for (int g = 0; g < groups; ++g) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a_off = ((kk / 4) * kDiagBox + (kk % 4) * 32) >> 4;
+                    const uint32_t b_off = ((kk / 4) * B_BOX + (kk % 4) * 32) >> 4;
+                    ptx::mma_ss(tmem, ad + a_off, bd + b_off, idesc, (g | kk) != 0);
+                }
+            }
+            ptx::mma_commit(bar);
+            volatile int never = 0;
+            const bool ok = ptx::mbar_wait(bar, 0, &never, wait_ns);
+            clocks[blockIdx.x] = ok ? clock64() - t0 : -1;
+            stop = 1;
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        float x0 = 0.001f * threadIdx.x, x1 = x0 + 0.25f, x2 = x0 + 0.5f, x3 = x0 + 0.75f;
+        uint32_t acc = 0;
+        for (int it = 0; it < (1 << 20) && !stop; ++it) {
+#pragma unroll
+            for (int r = 0; r < 64; ++r) {
+                if (BG == 0) {
+                    x0 = fmaf(x0, 0.999f, 0.001f);
+                    x1 = fmaf(x1, 0.999f, 0.001f);
+                    x2 = fmaf(x2, 0.999f, 0.001f);
+                    x3 = fmaf(x3, 0.999f, 0.001f);
+                } else if (BG == 1) {
+                    const float s0 = x0 * (x1 - 0.5f), s1 = x1 * (x2 - 0.25f);
+                    const float s2 = x2 * (x3 - 0.125f), s3 = x3 * (x0 - 0.0625f);
+                    acc ^= ptx::pack_bf16x2(s0, s1) ^ ptx::pack_bf16x2(s2, s3);
+                    x0 += 1e-3f;
+                    x1 += 1e-3f;
+                    x2 += 1e-3f;
+                    x3 += 1e-3f;
+                } else {
+                    const float p0 = ptx::ex2_approx(fmaf(x0, 0.01f, -1.f));
+                    const float p1 = ptx::ex2_approx(fmaf(x1, 0.01f, -1.f));
+                    x2 += p0;
+                    x3 += p1;
+                    x0 += 1e-3f;
+                    x1 += 1e-3f;
+                    acc ^= ptx::pack_bf16x2(p0, p1);
+                }
+            }
+        }
+        // the loop's results feed a store that no real value triggers, so it cannot be removed
+        if (__float_as_uint(x0 + x1 + x2 + x3) == 0x7fc00001u && acc == 0x12345u) clocks[blockIdx.x] = -3;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int BG>
+int launch_contended(long long* clocks, int ctas, int groups, unsigned long long wait_ns, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(skiparse_mma_contended_kernel<BG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kDiagSmem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    skiparse_mma_contended_kernel<BG><<<ctas, 384, kDiagSmem, st>>>(clocks, groups, wait_ns);
+    return static_cast<int>(cudaGetLastError());
+}
+
 }  // namespace
 
 static_assert(kDiagA + kDiagB + 1024 <= kDiagSmem, "diagnostic shared memory");
@@ -163,6 +272,9 @@ int launch_mma_rate(long long* clocks, int ctas, int pattern, int groups, unsign
         case 1: return launch_pattern<1>(clocks, ctas, groups, wait_ns, st);
         case 2: return launch_pattern<2>(clocks, ctas, groups, wait_ns, st);
         case 3: return launch_pattern<3>(clocks, ctas, groups, wait_ns, st);
+        case 4: return launch_contended<0>(clocks, ctas, groups, wait_ns, st);
+        case 5: return launch_contended<1>(clocks, ctas, groups, wait_ns, st);
+        case 6: return launch_contended<2>(clocks, ctas, groups, wait_ns, st);
         default: return static_cast<int>(cudaErrorInvalidValue);
     }
 }

@@ -210,7 +210,7 @@ int skiparse_debug_exp2(const float* x, float* y, long long n, int method,
 
 int skiparse_debug_mma_rate(int pattern, int groups, long long* clocks, int n_clocks,
                             skiparse_stream_t stream) {
-    if (pattern < 0 || pattern > 3 || groups < 1 || n_clocks < 1 || !clocks) return SKIPARSE_ERR_INVALID_ARG;
+    if (pattern < 0 || pattern > 6 || groups < 1 || n_clocks < 1 || !clocks) return SKIPARSE_ERR_INVALID_ARG;
     if (groups > 65536 || n_clocks > 4096) return SKIPARSE_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(clocks) & 7u) return SKIPARSE_ERR_MISALIGNED;
     const int e = skiparse::launch_mma_rate(clocks, n_clocks, pattern, groups, g_wait_limit_ns.load(), stream);

@@ -325,10 +325,12 @@ SKIPARSE_API int skiparse_debug_exp2(const float* x, float* y, long long n, int 
  * stream, as the attention kernels' MMA warp does, and writes the SM clocks from the first issue
  * to completion to clocks[cta] (-1 if its bounded wait ran out). Patterns: 0 = A and B in shared
  * memory, M = 128, N = 128; 1 = A in TMEM, M = N = 128; 2 = shared memory, N = 256;
- * 3 = shared memory, N = 64. One group is 8 x 2 x 128 x N x 16 FLOP; the nominal dense bf16 rate
- * of an SM is 8192 FLOP per clock.
+ * 3 = shared memory, N = 64; 4, 5, 6 = pattern 0 while 8 more warps of the CTA (2 per SM
+ * sub-partition) run independent FFMA chains (4), the backward's dS arithmetic (5: FADD, FMUL,
+ * bf16 pack) or the forward softmax's exponential loop (6) until the stream is done. One group
+ * is 8 x 2 x 128 x N x 16 FLOP; the nominal dense bf16 rate of an SM is 8192 FLOP per clock.
  *   clocks : device pointer to n_clocks int64, 8-byte aligned. 1 <= n_clocks <= 4096,
- *            1 <= groups <= 65536, 0 <= pattern <= 3.
+ *            1 <= groups <= 65536, 0 <= pattern <= 6.
  * Asynchronous on `stream`. Returns SKIPARSE_OK, SKIPARSE_ERR_INVALID_ARG, _UNSUPPORTED,
  * _MISALIGNED or SKIPARSE_ERR_CUDA.
  */

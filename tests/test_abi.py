@@ -150,7 +150,7 @@ def test_noalloc_backward_rejects_bad_arguments_before_any_cuda_call(L):
 
 
 def test_mma_rate_diagnostic_rejects_bad_arguments_synchronously(L):
-    assert L.skiparse_debug_mma_rate(4, 8, FAKE, 148, None) == 1
+    assert L.skiparse_debug_mma_rate(7, 8, FAKE, 148, None) == 1
     assert L.skiparse_debug_mma_rate(0, 0, FAKE, 148, None) == 1
     assert L.skiparse_debug_mma_rate(0, 8, 0, 148, None) == 1
     assert L.skiparse_debug_mma_rate(0, 1 << 20, FAKE, 148, None) == 2

@@ -29,7 +29,7 @@ def _rate(pattern: int, groups: int = 64):
     torch.cuda.synchronize()
     c = clocks.cpu().numpy()
     assert (c > 0).all(), "a CTA did not finish its MMA stream"
-    n = {0: 128, 1: 128, 2: 256, 3: 64}[pattern]
+    n = {0: 128, 1: 128, 2: 256, 3: 64, 4: 128, 5: 128, 6: 128}[pattern]
     flop = groups * 8 * 2.0 * 128 * n * 16
     return flop / np.median(c), np.median(c) / (groups * 8 * n / 128)
 
@@ -54,11 +54,24 @@ def test_n64_is_slower(cuda):
     assert per_clk < 0.9 * NOMINAL
 
 
+def test_issuer_starved_by_alu_bound_warps(cuda):
+    """The issuing thread shares an SM sub-partition with other warps. Warps running the
+    backward's dS arithmetic (FADD, FMUL, bf16 pack, no MUFU) leave it so few issue slots that
+    the tensor pipe runs at a small fraction of its rate; warps running the forward softmax's
+    exponential loop, which waits on the MUFU, cost it little. (Independent FFMA chains are
+    printed for reference: whether they starve the issuer depends on how the loop compiles.)"""
+    rates = {p: _rate(p)[0] / NOMINAL for p in (4, 5, 6)}
+    print("beside FFMA chains / dS arithmetic / exponential loop:",
+          " / ".join(f"{r:.3f}" for r in rates.values()), "of nominal")
+    assert rates[5] < 0.5
+    assert rates[6] >= 0.9
+
+
 def test_rejects_bad_arguments(cuda):
     from fixed_pattern_sparse_b200 import _lib
     L = _lib.lib()
     buf = torch.zeros(4, dtype=torch.int64, device="cuda")
-    assert L.skiparse_debug_mma_rate(4, 8, buf.data_ptr(), 4, None) == 1
+    assert L.skiparse_debug_mma_rate(7, 8, buf.data_ptr(), 4, None) == 1
     assert L.skiparse_debug_mma_rate(0, 0, buf.data_ptr(), 4, None) == 1
     assert L.skiparse_debug_mma_rate(0, 8, buf.data_ptr(), 5000, None) == 2
     assert L.skiparse_debug_mma_rate(0, 8, buf.data_ptr() + 4, 2, None) == 3
