@@ -65,3 +65,17 @@ def test_reference_arm_loads_only_the_oracle():
     assert line["impl"] == "reference" and line["value"] > 0
     check = json.loads(lines[-1])
     assert check == {"mods": [], "lib": False}
+
+
+def test_dram_traffic_entry_matches_the_current_forward_sources():
+    """bench.py reports `roofline.traffic` only for the forward kernel sources it was captured on
+    (keyed by their hash). An edit to those sources must come with a new one-pass capture of the
+    720p launch (dram__bytes_read.sum + dram__bytes_write.sum) and a new key; this test makes a
+    missing re-capture fail loudly instead of leaving the field silently null."""
+    h = bench.kernel_hash()
+    assert h in bench.KNOWN_TRAFFIC, (
+        f"forward sources hash {h} has no captured DRAM traffic: re-capture the 720p launch and key it")
+    # the captured bytes are the algorithmic ones: q, k, v read once and out written once (720p)
+    w = synth.WORKLOADS["720p"]
+    algorithmic = 4 * w.B * w.T * w.H * w.W * w.heads * w.d * 2
+    assert abs(bench.KNOWN_TRAFFIC[h] - algorithmic) / algorithmic < 0.01
